@@ -1,0 +1,495 @@
+// Host side of the C ABI declared in include/afd_ffn.h: argument validation, workspace
+// layout, TMA descriptor encoding and the launch sequence of one layer call
+// (route count -> route scan -> route scatter -> row gather -> W13 GEMM -> W2 GEMM).
+//
+// The FFN service of an AFD deployment receives activations and routing metadata,
+// computes the FFN output and returns it (vLLM AFD plugin, "FFN service"); FastAFD runs
+// the FFN side as one persistent kernel per layer (FastAFD, "Methodology / System
+// Design", item 3). Here the work is split into six stream-ordered launches that never
+// synchronise with the host.
+#include <cuda_runtime.h>
+#include <cuda.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <new>
+
+#include "afd_ffn.h"
+#include "gemm.cuh"
+#include "route.cuh"
+
+using namespace afd;
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn) return fn;
+  void* p = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess)
+    return nullptr;
+  fn = reinterpret_cast<EncodeTiledFn>(p);
+  return fn;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+}  // namespace
+
+struct afd_ffn_plan_s {
+  afd_ffn_config_t cfg;
+  afd_ffn_weights_t w;
+  int device = 0, num_sms = 0;
+  int G = 0, Tmax = 0, Rmax = 0, rpad = 0, num_chunks = 0;
+  void* ws = nullptr;
+  size_t ws_bytes = 0;
+  int32_t *slab_base, *info, *chunk_hist, *chunk_off, *group_count, *group_off, *mtile_off;
+  int32_t *tok_mt, *tok_need, *pos, *row_token, *row_k, *cnt;
+  float *row_w, *sa_t, *sh_t, *acc;
+  uint8_t *a_perm, *hq;
+  int* status;
+  CUtensorMap tm_a13, tm_w13, tm_a2, tm_w2;
+  bool timing = false, ev_valid = false;
+  cudaEvent_t ev[AFD_NUM_KERNELS + 1] = {};
+  unsigned long long wait_limit_ns = 1000000000ull;
+  int inject_stall = 0;
+  size_t scatter_smem = 0;
+};
+
+extern "C" {
+
+const char* afd_status_string(afd_status_t s) {
+  switch (s) {
+    case AFD_OK: return "AFD_OK";
+    case AFD_ERR_INVALID_ARGUMENT: return "AFD_ERR_INVALID_ARGUMENT";
+    case AFD_ERR_UNSUPPORTED: return "AFD_ERR_UNSUPPORTED";
+    case AFD_ERR_OUT_OF_MEMORY: return "AFD_ERR_OUT_OF_MEMORY";
+    case AFD_ERR_CUDA: return "AFD_ERR_CUDA";
+    case AFD_ERR_BAD_ROUTING: return "AFD_ERR_BAD_ROUTING";
+    case AFD_ERR_TIMEOUT: return "AFD_ERR_TIMEOUT";
+  }
+  return "unknown";
+}
+
+int32_t afd_ffn_kernels_per_layer(void) { return AFD_NUM_KERNELS; }
+
+afd_status_t afd_ffn_check_config(const afd_ffn_config_t* c) {
+  if (!c) return AFD_ERR_INVALID_ARGUMENT;
+  if (c->hidden < AFD_QBLOCK || c->hidden % AFD_QBLOCK) return AFD_ERR_INVALID_ARGUMENT;
+  if (c->intermediate < AFD_QBLOCK || c->intermediate % AFD_QBLOCK) return AFD_ERR_INVALID_ARGUMENT;
+  if (c->num_experts_global < 1 || c->expert_begin < 0 || c->num_local_experts < 0)
+    return AFD_ERR_INVALID_ARGUMENT;
+  if (static_cast<int64_t>(c->expert_begin) + c->num_local_experts > c->num_experts_global)
+    return AFD_ERR_INVALID_ARGUMENT;
+  if (c->has_shared_expert != 0 && c->has_shared_expert != 1) return AFD_ERR_INVALID_ARGUMENT;
+  if (c->num_local_experts + c->has_shared_expert < 1) return AFD_ERR_INVALID_ARGUMENT;
+  if (c->top_k < 1 || c->top_k > c->num_experts_global) return AFD_ERR_INVALID_ARGUMENT;
+  if (c->num_slabs < 1 || c->slab_capacity < 1) return AFD_ERR_INVALID_ARGUMENT;
+  // supported limits
+  if (c->hidden % 256) return AFD_ERR_UNSUPPORTED;   // W2 output tiles are 256 columns
+  if (c->top_k > AFD_MAX_TOP_K) return AFD_ERR_UNSUPPORTED;
+  if (c->num_slabs > AFD_MAX_SLABS) return AFD_ERR_UNSUPPORTED;
+  if (c->num_local_experts + c->has_shared_expert > AFD_MAX_GROUPS) return AFD_ERR_UNSUPPORTED;
+  if (c->slab_capacity >= (1 << 24)) return AFD_ERR_UNSUPPORTED;
+  const int64_t tmax = static_cast<int64_t>(c->num_slabs) * c->slab_capacity;
+  const int64_t kl = std::min(c->top_k, c->num_local_experts) + c->has_shared_expert;
+  if (tmax * c->top_k >= (int64_t{1} << 31) || tmax * kl + 256 >= (int64_t{1} << 31))
+    return AFD_ERR_UNSUPPORTED;
+  if ((tmax * kl + 256) * std::max(c->hidden, c->intermediate) >= (int64_t{1} << 40))
+    return AFD_ERR_UNSUPPORTED;
+  return AFD_OK;
+}
+
+static afd_status_t encode_2d(EncodeTiledFn enc, CUtensorMap* m, void* base, uint64_t inner,
+                              uint64_t rows) {
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {inner};
+  cuuint32_t box[2] = {128, 128};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, base, dims, strides, box, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? AFD_OK : AFD_ERR_CUDA;
+}
+
+static afd_status_t encode_3d(EncodeTiledFn enc, CUtensorMap* m, const void* base, uint64_t inner,
+                              uint64_t rows, uint64_t experts) {
+  cuuint64_t dims[3] = {inner, rows, experts};
+  cuuint64_t strides[2] = {inner, inner * rows};
+  cuuint32_t box[3] = {128, 128, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides,
+                   box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? AFD_OK : AFD_ERR_CUDA;
+}
+
+afd_status_t afd_ffn_plan(const afd_ffn_config_t* cfg, const afd_ffn_weights_t* weights,
+                          afd_ffn_plan_t* out) {
+  if (!out) return AFD_ERR_INVALID_ARGUMENT;
+  *out = nullptr;
+  afd_status_t st = afd_ffn_check_config(cfg);
+  if (st != AFD_OK) return st;
+  if (!weights || !weights->w13 || !weights->w2 || !weights->w13_scale || !weights->w2_scale)
+    return AFD_ERR_INVALID_ARGUMENT;
+  if (!aligned(weights->w13, 16) || !aligned(weights->w2, 16) || !aligned(weights->w13_scale, 4) ||
+      !aligned(weights->w2_scale, 4))
+    return AFD_ERR_INVALID_ARGUMENT;
+
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return AFD_ERR_UNSUPPORTED;
+  cudaDeviceProp prop;
+  if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return AFD_ERR_CUDA;
+  if (prop.major != 10 || prop.minor != 0) return AFD_ERR_UNSUPPORTED;
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return AFD_ERR_CUDA;
+  // The GEMM kernels split the block's registers between warpgroups with setmaxnreg; that
+  // is only safe when the block is launched with exactly the budget the split assumes.
+  for (int epi = 0; epi < 2; ++epi) {
+    cudaFuncAttributes fa;
+    cudaError_t e = epi == 0 ? cudaFuncGetAttributes(&fa, grouped_gemm_kernel<EPI_SWIGLU>)
+                             : cudaFuncGetAttributes(&fa, grouped_gemm_kernel<EPI_COMBINE>);
+    if (e != cudaSuccess) return AFD_ERR_CUDA;
+    if (fa.numRegs != kLaunchRegs || fa.maxThreadsPerBlock < kGemmThreads) return AFD_ERR_UNSUPPORTED;
+  }
+
+  afd_ffn_plan_s* P = new (std::nothrow) afd_ffn_plan_s();
+  if (!P) return AFD_ERR_OUT_OF_MEMORY;
+  P->cfg = *cfg;
+  P->w = *weights;
+  P->device = dev;
+  P->num_sms = prop.multiProcessorCount;
+  const int H = cfg->hidden, I = cfg->intermediate, K = cfg->top_k;
+  const int El = cfg->num_local_experts, S = cfg->has_shared_expert;
+  P->G = El + S;
+  P->Tmax = cfg->num_slabs * cfg->slab_capacity;
+  P->Rmax = P->Tmax * (std::min(K, El) + S);
+  P->rpad = ((P->Rmax + 128 + 127) / 128) * 128;
+  P->num_chunks = (P->Tmax + kChunkTokens - 1) / kChunkTokens;
+  const int El1 = std::max(El, 1);
+
+  // workspace layout
+  size_t off = 0;
+  auto take = [&](size_t bytes, size_t align) {
+    off = (off + align - 1) / align * align;
+    size_t o = off;
+    off += bytes;
+    return o;
+  };
+  const size_t o_slab_base = take(sizeof(int32_t) * (cfg->num_slabs + 1), 16);
+  const size_t o_info = take(sizeof(int32_t) * 16, 16);
+  const size_t o_status = take(sizeof(int32_t) * 4, 16);
+  const size_t o_chunk_hist = take(sizeof(int32_t) * P->num_chunks * El1, 16);
+  const size_t o_chunk_off = take(sizeof(int32_t) * P->num_chunks * El1, 16);
+  const size_t o_group_count = take(sizeof(int32_t) * (P->G + 1), 16);
+  const size_t o_group_off = take(sizeof(int32_t) * (P->G + 1), 16);
+  const size_t o_mtile_off = take(sizeof(int32_t) * (P->G + 1), 16);
+  const size_t o_tok_mt = take(sizeof(int32_t) * P->Tmax, 16);
+  const size_t o_tok_need = take(sizeof(int32_t) * P->Tmax, 16);
+  const size_t o_pos = take(sizeof(int32_t) * static_cast<size_t>(P->Tmax) * K, 16);
+  const size_t o_row_token = take(sizeof(int32_t) * P->rpad, 16);
+  const size_t o_row_k = take(sizeof(int32_t) * P->rpad, 16);
+  const size_t o_row_w = take(sizeof(float) * P->rpad, 16);
+  const size_t o_a_perm = take(static_cast<size_t>(P->rpad) * H, 1024);
+  const size_t o_sa_t = take(sizeof(float) * static_cast<size_t>(H / 128) * P->rpad, 256);
+  const size_t o_hq = take(static_cast<size_t>(P->rpad) * I, 1024);
+  const size_t o_sh_t = take(sizeof(float) * static_cast<size_t>(I / 128) * P->rpad, 256);
+  const size_t o_acc = take(sizeof(float) * static_cast<size_t>(P->Tmax) * H, 256);
+  const size_t o_cnt = take(sizeof(int32_t) * static_cast<size_t>(P->Tmax) * (H / 256), 256);
+  P->ws_bytes = take(0, 256);
+
+  if (cudaMalloc(&P->ws, P->ws_bytes) != cudaSuccess) {
+    cudaGetLastError();
+    delete P;
+    return AFD_ERR_OUT_OF_MEMORY;
+  }
+  if (cudaMemset(P->ws, 0, P->ws_bytes) != cudaSuccess) {
+    cudaFree(P->ws);
+    delete P;
+    return AFD_ERR_CUDA;
+  }
+  uint8_t* b = static_cast<uint8_t*>(P->ws);
+  P->slab_base = reinterpret_cast<int32_t*>(b + o_slab_base);
+  P->info = reinterpret_cast<int32_t*>(b + o_info);
+  P->status = reinterpret_cast<int*>(b + o_status);
+  P->chunk_hist = reinterpret_cast<int32_t*>(b + o_chunk_hist);
+  P->chunk_off = reinterpret_cast<int32_t*>(b + o_chunk_off);
+  P->group_count = reinterpret_cast<int32_t*>(b + o_group_count);
+  P->group_off = reinterpret_cast<int32_t*>(b + o_group_off);
+  P->mtile_off = reinterpret_cast<int32_t*>(b + o_mtile_off);
+  P->tok_mt = reinterpret_cast<int32_t*>(b + o_tok_mt);
+  P->tok_need = reinterpret_cast<int32_t*>(b + o_tok_need);
+  P->pos = reinterpret_cast<int32_t*>(b + o_pos);
+  P->row_token = reinterpret_cast<int32_t*>(b + o_row_token);
+  P->row_k = reinterpret_cast<int32_t*>(b + o_row_k);
+  P->row_w = reinterpret_cast<float*>(b + o_row_w);
+  P->a_perm = b + o_a_perm;
+  P->sa_t = reinterpret_cast<float*>(b + o_sa_t);
+  P->hq = b + o_hq;
+  P->sh_t = reinterpret_cast<float*>(b + o_sh_t);
+  P->acc = reinterpret_cast<float*>(b + o_acc);
+  P->cnt = reinterpret_cast<int32_t*>(b + o_cnt);
+
+  const int E = P->G;
+  st = encode_2d(enc, &P->tm_a13, P->a_perm, H, P->rpad);
+  if (st == AFD_OK) st = encode_3d(enc, &P->tm_w13, weights->w13, H, 2 * static_cast<uint64_t>(I), E);
+  if (st == AFD_OK) st = encode_2d(enc, &P->tm_a2, P->hq, I, P->rpad);
+  if (st == AFD_OK) st = encode_3d(enc, &P->tm_w2, weights->w2, I, H, E);
+  if (st != AFD_OK) {
+    cudaFree(P->ws);
+    delete P;
+    return st;
+  }
+  P->scatter_smem = sizeof(int32_t) * (static_cast<size_t>(kRouteWarps) * El1 + kRouteWarps * 32 * K);
+  if (cudaFuncSetAttribute(grouped_gemm_kernel<EPI_SWIGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(gemm_smem_bytes(EPI_SWIGLU))) != cudaSuccess ||
+      cudaFuncSetAttribute(grouped_gemm_kernel<EPI_COMBINE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(gemm_smem_bytes(EPI_COMBINE))) != cudaSuccess ||
+      cudaFuncSetAttribute(route_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(std::max<size_t>(P->scatter_smem, 1))) != cudaSuccess) {
+    cudaGetLastError();
+    cudaFree(P->ws);
+    delete P;
+    return AFD_ERR_CUDA;
+  }
+  for (int i = 0; i <= AFD_NUM_KERNELS; ++i) cudaEventCreate(&P->ev[i]);
+  *out = P;
+  return AFD_OK;
+}
+
+void afd_ffn_destroy(afd_ffn_plan_t P) {
+  if (!P) return;
+  cudaDeviceSynchronize();
+  for (int i = 0; i <= AFD_NUM_KERNELS; ++i)
+    if (P->ev[i]) cudaEventDestroy(P->ev[i]);
+  if (P->ws) cudaFree(P->ws);
+  delete P;
+}
+
+afd_status_t afd_ffn_get_info(afd_ffn_plan_t P, afd_ffn_plan_info_t* info) {
+  if (!P || !info) return AFD_ERR_INVALID_ARGUMENT;
+  info->num_groups = P->G;
+  info->max_tokens = P->Tmax;
+  info->max_rows = P->Rmax;
+  info->num_sms = P->num_sms;
+  info->workspace_bytes = static_cast<int64_t>(P->ws_bytes);
+  return AFD_OK;
+}
+
+static void fill_route_params(afd_ffn_plan_t P, const int32_t* d_counts, RouteParams& rp) {
+  const afd_ffn_config_t& c = P->cfg;
+  rp.counts = d_counts;
+  rp.M = c.num_slabs;
+  rp.cap = c.slab_capacity;
+  rp.K = c.top_k;
+  rp.H = c.hidden;
+  rp.e0 = c.expert_begin;
+  rp.El = c.num_local_experts;
+  rp.Eg = c.num_experts_global;
+  rp.S = c.has_shared_expert;
+  rp.G = P->G;
+  rp.num_chunks = P->num_chunks;
+  rp.rpad = P->rpad;
+  rp.slab_base = P->slab_base;
+  rp.info = P->info;
+  rp.chunk_hist = P->chunk_hist;
+  rp.chunk_off = P->chunk_off;
+  rp.group_count = P->group_count;
+  rp.group_off = P->group_off;
+  rp.mtile_off = P->mtile_off;
+  rp.tok_mt = P->tok_mt;
+  rp.tok_need = P->tok_need;
+  rp.pos = P->pos;
+  rp.row_token = P->row_token;
+  rp.row_k = P->row_k;
+  rp.row_w = P->row_w;
+  rp.a_perm = P->a_perm;
+  rp.sa_t = P->sa_t;
+  rp.status = P->status;
+}
+
+static void fill_gemm_params(afd_ffn_plan_t P, int epi, GemmParams& gp) {
+  const afd_ffn_config_t& c = P->cfg;
+  memset(&gp, 0, sizeof(gp));
+  gp.group_off = P->group_off;
+  gp.mtile_off = P->mtile_off;
+  gp.G = P->G;
+  gp.rpad = P->rpad;
+  gp.I = c.intermediate;
+  gp.H = c.hidden;
+  gp.status = P->status;
+  gp.wait_limit_ns = P->wait_limit_ns;
+  if (epi == EPI_SWIGLU) {
+    gp.n_tiles = c.intermediate / 128;
+    gp.num_kb = c.hidden / 128;
+    gp.sa_t = P->sa_t;
+    gp.w_scale = P->w.w13_scale;
+    gp.ws_rows = 2 * c.intermediate / 128;
+    gp.hq = P->hq;
+    gp.sh_t = P->sh_t;
+    gp.inject_stall = P->inject_stall;
+  } else {
+    gp.n_tiles = c.hidden / 256;
+    gp.num_kb = c.intermediate / 128;
+    gp.sa_t = P->sh_t;
+    gp.w_scale = P->w.w2_scale;
+    gp.ws_rows = c.hidden / 128;
+    gp.row_token = P->row_token;
+    gp.row_w = P->row_w;
+    gp.tok_mt = P->tok_mt;
+    gp.tok_need = P->tok_need;
+    gp.acc = P->acc;
+    gp.cnt = P->cnt;
+  }
+}
+
+afd_status_t afd_ffn_layer(afd_ffn_plan_t P, const afd_slab_t* slabs, const int32_t* d_counts,
+                           afd_stream_t stream_) {
+  if (!P || !slabs || !d_counts) return AFD_ERR_INVALID_ARGUMENT;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  const afd_ffn_config_t& c = P->cfg;
+  SlabTable tab;
+  YTable ytab;
+  memset(&tab, 0, sizeof(tab));
+  memset(&ytab, 0, sizeof(ytab));
+  for (int m = 0; m < c.num_slabs; ++m) {
+    const afd_slab_t& s = slabs[m];
+    if (!s.x || !s.x_scale || !s.topk_ids || !s.topk_weights || !s.y) return AFD_ERR_INVALID_ARGUMENT;
+    if (!aligned(s.x, 16) || !aligned(s.y, 16) || !aligned(s.x_scale, 4) || !aligned(s.topk_ids, 4) ||
+        !aligned(s.topk_weights, 4))
+      return AFD_ERR_INVALID_ARGUMENT;
+    tab.x[m] = static_cast<const uint8_t*>(s.x);
+    tab.xs[m] = s.x_scale;
+    tab.ids[m] = s.topk_ids;
+    tab.w[m] = s.topk_weights;
+    tab.y[m] = static_cast<__nv_bfloat16*>(s.y);
+    ytab.y[m] = static_cast<__nv_bfloat16*>(s.y);
+  }
+  RouteParams rp;
+  fill_route_params(P, d_counts, rp);
+  GemmParams g13, g2;
+  fill_gemm_params(P, EPI_SWIGLU, g13);
+  fill_gemm_params(P, EPI_COMBINE, g2);
+  P->inject_stall = 0;
+
+  const bool tm = P->timing;
+  if (tm) cudaEventRecord(P->ev[0], stream);
+  route_count_kernel<<<P->num_chunks, kRouteThreads, 0, stream>>>(rp, tab);
+  if (tm) cudaEventRecord(P->ev[1], stream);
+  route_scan_kernel<<<1, 1024, 0, stream>>>(rp);
+  if (tm) cudaEventRecord(P->ev[2], stream);
+  route_scatter_kernel<<<P->num_chunks, kRouteThreads, P->scatter_smem, stream>>>(rp, tab);
+  if (tm) cudaEventRecord(P->ev[3], stream);
+  gather_rows_kernel<<<P->num_sms * 4, kRouteThreads, 0, stream>>>(rp, tab);
+  if (tm) cudaEventRecord(P->ev[4], stream);
+  grouped_gemm_kernel<EPI_SWIGLU><<<P->num_sms, kGemmThreads, gemm_smem_bytes(EPI_SWIGLU), stream>>>(
+      g13, P->tm_a13, P->tm_w13, ytab);
+  if (tm) cudaEventRecord(P->ev[5], stream);
+  grouped_gemm_kernel<EPI_COMBINE><<<P->num_sms, kGemmThreads, gemm_smem_bytes(EPI_COMBINE), stream>>>(
+      g2, P->tm_a2, P->tm_w2, ytab);
+  if (tm) cudaEventRecord(P->ev[6], stream);
+  P->ev_valid = tm;
+  if (cudaGetLastError() != cudaSuccess) return AFD_ERR_CUDA;
+  return AFD_OK;
+}
+
+afd_status_t afd_ffn_get_status(afd_ffn_plan_t P, afd_stream_t stream, int32_t* word) {
+  if (!P) return AFD_ERR_INVALID_ARGUMENT;
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return AFD_ERR_CUDA;
+  int32_t v = 0;
+  if (cudaMemcpy(&v, P->status, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return AFD_ERR_CUDA;
+  if (cudaMemset(P->status, 0, sizeof(v)) != cudaSuccess) return AFD_ERR_CUDA;
+  if (word) *word = v;
+  if (v & AFD_STATUS_TIMEOUT) return AFD_ERR_TIMEOUT;
+  if (v & (AFD_STATUS_BAD_ROUTING | AFD_STATUS_BAD_COUNT)) return AFD_ERR_BAD_ROUTING;
+  return AFD_OK;
+}
+
+static afd_status_t d2h(void* dst, const void* src, size_t bytes) {
+  if (!dst || bytes == 0) return AFD_OK;
+  return cudaMemcpy(dst, src, bytes, cudaMemcpyDeviceToHost) == cudaSuccess ? AFD_OK : AFD_ERR_CUDA;
+}
+
+afd_status_t afd_ffn_read_routing(afd_ffn_plan_t P, afd_stream_t stream, int32_t* num_tokens,
+                                  int32_t* num_rows, int32_t* counts, int32_t* offsets,
+                                  int32_t* row_token, int32_t* row_k, float* row_weight,
+                                  int32_t* pos) {
+  if (!P) return AFD_ERR_INVALID_ARGUMENT;
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return AFD_ERR_CUDA;
+  int32_t info[4];
+  if (cudaMemcpy(info, P->info, sizeof(info), cudaMemcpyDeviceToHost) != cudaSuccess) return AFD_ERR_CUDA;
+  const int T = info[0], R = info[1];
+  if (num_tokens) *num_tokens = T;
+  if (num_rows) *num_rows = R;
+  afd_status_t s = AFD_OK;
+  if (s == AFD_OK) s = d2h(counts, P->group_count, sizeof(int32_t) * P->G);
+  if (s == AFD_OK) s = d2h(offsets, P->group_off, sizeof(int32_t) * (P->G + 1));
+  if (s == AFD_OK) s = d2h(row_token, P->row_token, sizeof(int32_t) * R);
+  if (s == AFD_OK) s = d2h(row_k, P->row_k, sizeof(int32_t) * R);
+  if (s == AFD_OK) s = d2h(row_weight, P->row_w, sizeof(float) * R);
+  if (s == AFD_OK) s = d2h(pos, P->pos, sizeof(int32_t) * static_cast<size_t>(T) * P->cfg.top_k);
+  return s;
+}
+
+afd_status_t afd_ffn_read_intermediate(afd_ffn_plan_t P, afd_stream_t stream, uint8_t* h_codes,
+                                       float* h_scales) {
+  if (!P) return AFD_ERR_INVALID_ARGUMENT;
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return AFD_ERR_CUDA;
+  int32_t info[4];
+  if (cudaMemcpy(info, P->info, sizeof(info), cudaMemcpyDeviceToHost) != cudaSuccess) return AFD_ERR_CUDA;
+  const int R = info[1];
+  const int I = P->cfg.intermediate;
+  afd_status_t s = d2h(h_codes, P->hq, static_cast<size_t>(R) * I);
+  if (s == AFD_OK && h_scales && R > 0) {
+    // stored transposed [I/128][rpad]; return row-major [R][I/128]
+    const int nb = I / 128;
+    float* tmp = static_cast<float*>(malloc(sizeof(float) * static_cast<size_t>(nb) * R));
+    if (!tmp) return AFD_ERR_OUT_OF_MEMORY;
+    for (int j = 0; j < nb && s == AFD_OK; ++j)
+      s = d2h(tmp + static_cast<size_t>(j) * R, P->sh_t + static_cast<size_t>(j) * P->rpad,
+              sizeof(float) * R);
+    for (int r = 0; r < R; ++r)
+      for (int j = 0; j < nb; ++j) h_scales[static_cast<size_t>(r) * nb + j] = tmp[static_cast<size_t>(j) * R + r];
+    free(tmp);
+  }
+  return s;
+}
+
+afd_status_t afd_ffn_set_timing(afd_ffn_plan_t P, int32_t enable) {
+  if (!P) return AFD_ERR_INVALID_ARGUMENT;
+  P->timing = enable != 0;
+  return AFD_OK;
+}
+
+afd_status_t afd_ffn_get_kernel_times(afd_ffn_plan_t P, float* ms) {
+  if (!P || !ms) return AFD_ERR_INVALID_ARGUMENT;
+  if (!P->ev_valid) return AFD_ERR_INVALID_ARGUMENT;
+  if (cudaEventSynchronize(P->ev[AFD_NUM_KERNELS]) != cudaSuccess) return AFD_ERR_CUDA;
+  for (int i = 0; i < AFD_NUM_KERNELS; ++i)
+    if (cudaEventElapsedTime(&ms[i], P->ev[i], P->ev[i + 1]) != cudaSuccess) return AFD_ERR_CUDA;
+  return AFD_OK;
+}
+
+afd_status_t afd_ffn_set_wait_limit(afd_ffn_plan_t P, int64_t limit_ns) {
+  if (!P || limit_ns <= 0) return AFD_ERR_INVALID_ARGUMENT;
+  P->wait_limit_ns = static_cast<unsigned long long>(limit_ns);
+  return AFD_OK;
+}
+
+afd_status_t afd_ffn_inject_stall(afd_ffn_plan_t P, int32_t enable) {
+  if (!P) return AFD_ERR_INVALID_ARGUMENT;
+  P->inject_stall = enable != 0;
+  return AFD_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,434 @@
+// Persistent block-FP8 grouped GEMM for sm_100a (tcgen05 + TMEM + TMA), used for both
+// expert projections of the FFN-pool layer (FastAFD, "Methodology / System Design",
+// item 3: "block-FP8 grouped GEMMs, activation and push-back").
+//
+// Tile: 128 routed rows of one expert x 256 output columns, K in blocks of 128 (the
+// quantisation block). Each 128-wide K block is one tcgen05 partial product
+// (4 x kind::f8f6f4 MMAs of K=32) into one of two TMEM buffers; the epilogue warps read
+// the partial, multiply it by (row scale x weight-block scale) and accumulate in fp32
+// registers ("software promotion": the scales are arbitrary fp32, so they cannot ride on
+// the hardware's UE8M0 block-scale path).
+//
+// Warp roles (384 threads): warp 0 issues TMA loads, warp 1 owns TMEM and issues MMAs,
+// warps 2..3 idle, warps 4..11 are the epilogue (two per TMEM lane quadrant, splitting
+// the columns).
+//
+// Epilogues:
+//   SWIGLU   (W13) columns are [gate 128 | up 128] of intermediate block nt; h = silu(g)*u
+//            is requantised to e4m3 per (row, 128 channels) and stored with its scale.
+//   COMBINE  (W2)  the row's result times its top-K weight is added (fp32 reductions in
+//            L2) into the token's accumulator; the last contribution to a (token, 256
+//            columns) piece converts it to bf16, writes it into the token's slab row and
+//            clears the accumulator and counter for the next call.
+#pragma once
+
+#include "ptx.cuh"
+#include "route.cuh"
+
+namespace afd {
+
+constexpr int kStages = 4;
+constexpr int kBN = 256;
+constexpr int kBK = 128;
+constexpr int kGemmThreads = 384;
+// Register split: the block launches with kLaunchRegs per thread; warpgroup 0 (TMA, MMA,
+// two idle warps) drops to kProducerRegs and the two epilogue warpgroups rise to
+// kEpilogueRegs. 128*40 + 256*232 == 384*168, so the increase never waits for registers
+// the block does not own; the host refuses to launch if the compiled count differs.
+constexpr int kLaunchRegs = 168;
+constexpr int kProducerRegs = 40;
+constexpr int kEpilogueRegs = 232;
+static_assert(128 * kProducerRegs + 256 * kEpilogueRegs <= kGemmThreads * kLaunchRegs,
+              "register split exceeds the launch allocation");
+constexpr int kEpiWarps = 8;
+constexpr uint32_t kABytes = kTileM * kBK;   // 16 KiB
+constexpr uint32_t kBBytes = kBN * kBK;      // 32 KiB
+constexpr uint32_t kStageBytes = kABytes + kBBytes;
+constexpr int kStgStride = 20;               // floats per staging row (16 + 4 pad)
+constexpr uint32_t kTmemCols = 512;          // two 256-column fp32 partial buffers
+
+enum EpiKind { EPI_SWIGLU = 0, EPI_COMBINE = 1 };
+
+struct YTable {
+  __nv_bfloat16* y[AFD_MAX_SLABS];
+};
+
+struct GemmParams {
+  const int32_t* group_off;   // [G+1] first row of each group
+  const int32_t* mtile_off;   // [G+1] first m-tile of each group
+  int G;
+  int n_tiles;                // 256-column tiles per m-tile
+  int num_kb;                 // K blocks of 128
+  const float* sa_t;          // A scales, [num_kb][rpad]
+  int rpad;
+  const float* w_scale;       // [E][ws_rows][num_kb]
+  int ws_rows;
+  int I;
+  int H;
+  // SWIGLU epilogue outputs
+  uint8_t* hq;                // [rpad][I]
+  float* sh_t;                // [I/128][rpad]
+  // COMBINE epilogue inputs/outputs
+  const int32_t* row_token;
+  const float* row_w;
+  const int32_t* tok_mt;
+  const int32_t* tok_need;
+  float* acc;                 // [Tmax][H] fp32, zero between calls
+  int32_t* cnt;               // [Tmax][H/256], zero between calls
+  int* status;
+  unsigned long long wait_limit_ns;
+  int inject_stall;
+};
+
+struct GemmSmem {
+  uint64_t full[kStages];
+  uint64_t empty[kStages];
+  uint64_t tfull[2];
+  uint64_t tempty[2];
+  uint64_t pair[4];           // SWIGLU: amax exchange between the two warps of a quadrant
+  uint32_t tmem_base;
+  int abort_flag;
+  float amax[2][2][kTileM];
+  int32_t mtile[AFD_MAX_GROUPS + 1];
+};
+
+constexpr size_t kGemmSmemTiles = static_cast<size_t>(kStages) * kStageBytes;
+constexpr size_t kStgBytes = static_cast<size_t>(kEpiWarps) * 32 * kStgStride * sizeof(float);
+
+__host__ __device__ constexpr size_t gemm_smem_bytes(int epi) {
+  return 1024 + kGemmSmemTiles + sizeof(GemmSmem) + (epi == EPI_COMBINE ? kStgBytes : 0);
+}
+
+// A wait that ignores the abort flag; used only to drain copies/MMAs already in flight.
+__device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+  const uint32_t a = smem_u32(bar);
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(a, parity)) {
+    if (globaltimer_ns() - t0 > limit_ns) return;
+  }
+}
+
+struct TileCoord {
+  int e, row0, rows, nt;
+};
+
+__device__ __forceinline__ TileCoord decode_tile(int tile, int n_tiles, const int32_t* s_mtile,
+                                                 int G, const int32_t* group_off) {
+  TileCoord c;
+  const int mt = tile / n_tiles;
+  c.nt = tile - mt * n_tiles;
+  int lo = 0, hi = G - 1;               // last group whose first m-tile is <= mt
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (s_mtile[mid] <= mt) lo = mid; else hi = mid - 1;
+  }
+  c.e = lo;
+  const int g0 = group_off[lo], g1 = group_off[lo + 1];
+  c.row0 = g0 + (mt - s_mtile[lo]) * kTileM;
+  c.rows = min(kTileM, g1 - c.row0);
+  return c;
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    grouped_gemm_kernel(const __grid_constant__ GemmParams p,
+                        const __grid_constant__ CUtensorMap tm_a,
+                        const __grid_constant__ CUtensorMap tm_b,
+                        const __grid_constant__ YTable ytab) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  uint8_t* sA = base;
+  uint8_t* sB = base + kStages * kABytes;
+  GemmSmem& S = *reinterpret_cast<GemmSmem*>(base + kGemmSmemTiles);
+  float* stg = reinterpret_cast<float*>(base + kGemmSmemTiles + sizeof(GemmSmem));
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  volatile int* abort_flag = &S.abort_flag;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&S.full[s], 1);
+      mbar_init(&S.empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&S.tfull[b], 1);
+      mbar_init(&S.tempty[b], kEpiWarps);
+    }
+    for (int i = 0; i < 4; ++i) mbar_init(&S.pair[i], 64);
+    S.abort_flag = 0;
+    fence_mbar_init();
+  }
+  for (int i = threadIdx.x; i <= p.G; i += blockDim.x) S.mtile[i] = p.mtile_off[i];
+  if (warp == 1) {
+    tmem_alloc(&S.tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = S.tmem_base;
+  const int total_tiles = S.mtile[p.G] * p.n_tiles;
+
+  if (warp < 4) {
+    // each role's code sits inside the branch that sets its register budget
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kProducerRegs));
+    if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_a);
+      tma_prefetch_desc(&tm_b);
+      const uint64_t pol_a = policy_evict_last();
+      const uint64_t pol_b = policy_evict_last();
+      int it = 0;
+      bool ok = true;
+      int skipped = -1;
+      for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
+        const TileCoord c = decode_tile(tile, p.n_tiles, S.mtile, p.G, p.group_off);
+        for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
+          const int s = it % kStages;
+          const uint32_t ph = (it / kStages) & 1;
+          if (!mbar_wait(&S.empty[s], ph ^ 1, abort_flag, p.status, p.wait_limit_ns)) {
+            ok = false;
+            break;
+          }
+          if (p.inject_stall && blockIdx.x == 0 && it == 0) {
+            skipped = it;       // test hook: never fill this stage
+            continue;
+          }
+          mbar_arrive_expect_tx(&S.full[s], kStageBytes);
+          tma_load_2d(sA + s * kABytes, &tm_a, &S.full[s], kb * kBK, c.row0, pol_a);
+          uint8_t* b = sB + s * kBBytes;
+          if (EPI == EPI_SWIGLU) {
+            tma_load_3d(b, &tm_b, &S.full[s], kb * kBK, c.nt * 128, c.e, pol_b);
+            tma_load_3d(b + kBBytes / 2, &tm_b, &S.full[s], kb * kBK, p.I + c.nt * 128, c.e, pol_b);
+          } else {
+            tma_load_3d(b, &tm_b, &S.full[s], kb * kBK, c.nt * kBN, c.e, pol_b);
+            tma_load_3d(b + kBBytes / 2, &tm_b, &S.full[s], kb * kBK, c.nt * kBN + 128, c.e, pol_b);
+          }
+        }
+      }
+      if (!ok) {
+        // wait (bounded) for the copies this thread issued that may still be landing
+        for (int j = max(0, it - kStages); j < it; ++j) {
+          if (j == skipped) continue;
+          mbar_wait_drain(&S.full[j % kStages], (j / kStages) & 1, p.wait_limit_ns);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_e4m3_f32(kTileM, kBN);
+      int it = 0, kbg = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
+        for (int kb = 0; kb < p.num_kb; ++kb, ++it, ++kbg) {
+          const int s = it % kStages;
+          const uint32_t ph = (it / kStages) & 1;
+          if (!mbar_wait(&S.full[s], ph, abort_flag, p.status, p.wait_limit_ns)) {
+            ok = false;
+            break;
+          }
+          const int b = kbg & 1;
+          const uint32_t tph = (kbg >> 1) & 1;
+          if (!mbar_wait(&S.tempty[b], tph ^ 1, abort_flag, p.status, p.wait_limit_ns)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t d = tmem_base + b * kBN;
+          const uint64_t a0 = sdesc_k_sw128(smem_u32(sA + s * kABytes));
+          const uint64_t b0 = sdesc_k_sw128(smem_u32(sB + s * kBBytes));
+#pragma unroll
+          for (int k = 0; k < kBK / 32; ++k)
+            umma_e4m3(d, a0 + 2 * k, b0 + 2 * k, idesc, k > 0 ? 1u : 0u);
+          umma_commit(&S.empty[s]);
+          umma_commit(&S.tfull[b]);
+        }
+      }
+      if (!ok && kbg > 0) {
+        const int last = kbg - 1;
+        mbar_wait_drain(&S.tfull[last & 1], (last >> 1) & 1, p.wait_limit_ns);
+      }
+    }
+    }
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kEpilogueRegs));
+    // ------------------------------------------------------------------ epilogue
+    const int ew = warp - 4;
+    const int half = ew >> 2;
+    const int q = warp & 3;                 // TMEM lane quadrant this warp may access
+    const int trow = 32 * q + lane;
+    const uint32_t tq = tmem_base + (static_cast<uint32_t>(32 * q) << 16);
+    int kbg = 0, titer = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x, ++titer) {
+      const TileCoord c = decode_tile(tile, p.n_tiles, S.mtile, p.G, p.group_off);
+      const int grow = c.row0 + trow;
+      const bool valid = trow < c.rows;
+      const float* wsb = p.w_scale + static_cast<size_t>(c.e) * p.ws_rows * p.num_kb;
+      int rs0, rs1, c0, c1;
+      if (EPI == EPI_SWIGLU) {
+        rs0 = c.nt;
+        rs1 = p.I / 128 + c.nt;
+        c0 = 64 * half;
+        c1 = 128 + 64 * half;
+      } else {
+        rs0 = rs1 = 2 * c.nt + half;
+        c0 = 128 * half;
+        c1 = 128 * half + 64;
+      }
+      const float* ws0 = wsb + static_cast<size_t>(rs0) * p.num_kb;
+      const float* ws1 = wsb + static_cast<size_t>(rs1) * p.num_kb;
+      float acc[128];
+#pragma unroll
+      for (int i = 0; i < 128; ++i) acc[i] = 0.f;
+      for (int kb = 0; kb < p.num_kb; ++kb, ++kbg) {
+        const float sa = p.sa_t[static_cast<size_t>(kb) * p.rpad + grow];
+        const float s0 = sa * __ldg(ws0 + kb);
+        const float s1 = sa * __ldg(ws1 + kb);
+        const int b = kbg & 1;
+        const uint32_t tph = (kbg >> 1) & 1;
+        int got = 1;
+        if (lane == 0) got = mbar_wait(&S.tfull[b], tph, abort_flag, p.status, p.wait_limit_ns);
+        got = __shfl_sync(0xffffffffu, got, 0);
+        if (!got) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t tb = tq + b * kBN;
+        {
+          float v[32], w[32];
+          tmem_ld32(tb + c0, v);
+          tmem_ld32(tb + c0 + 32, w);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) acc[i] = fmaf(v[i], s0, acc[i]);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) acc[32 + i] = fmaf(w[i], s0, acc[32 + i]);
+        }
+        {
+          float v[32], w[32];
+          tmem_ld32(tb + c1, v);
+          tmem_ld32(tb + c1 + 32, w);
+          tmem_wait_ld();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&S.tempty[b]);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) acc[64 + i] = fmaf(v[i], s1, acc[64 + i]);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) acc[96 + i] = fmaf(w[i], s1, acc[96 + i]);
+        }
+      }
+      if (!ok) break;
+
+      if (EPI == EPI_SWIGLU) {
+        // h = silu(g) * u on this thread's 64 channels; block amax shared with the partner
+        // warp that holds the other 64 channels of the same rows
+        float amax = 0.f;
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+          const float g = acc[i];
+          const float h = (g / (1.0f + expf(-g))) * acc[64 + i];
+          acc[i] = h;
+          amax = fmaxf(amax, fabsf(h));
+        }
+        float* ax = &S.amax[titer & 1][0][0];
+        ax[half * kTileM + trow] = amax;
+        mbar_arrive(&S.pair[q]);
+        if (!mbar_wait(&S.pair[q], titer & 1, abort_flag, p.status, p.wait_limit_ns)) {
+          ok = false;
+          break;
+        }
+        amax = fmaxf(amax, ax[(half ^ 1) * kTileM + trow]);
+        const float sc = amax > 0.f ? amax / 448.0f : 1.0f;
+        if (valid) {
+          uint4 out[4];
+          uint16_t* o16 = reinterpret_cast<uint16_t*>(out);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o16[i] = pack_e4m3x2(acc[2 * i] / sc, acc[2 * i + 1] / sc);
+          uint4* dst = reinterpret_cast<uint4*>(p.hq + static_cast<size_t>(grow) * p.I +
+                                                c.nt * 128 + 64 * half);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) dst[j] = out[j];
+          if (half == 0) p.sh_t[static_cast<size_t>(c.nt) * p.rpad + grow] = sc;
+        }
+      } else {
+        // weighted combine: fp32 reductions into the token accumulator, staged through
+        // shared memory so that each reduction covers 128 contiguous bytes of one row
+        int g = -1;
+        float wgt = 0.f;
+        if (valid) {
+          g = p.row_token[grow];
+          wgt = p.row_w[grow];
+        }
+        float* sw = stg + ew * 32 * kStgStride;
+        const int col0 = c.nt * kBN + half * 128;
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            float4 v = make_float4(acc[16 * ch + 4 * j] * wgt, acc[16 * ch + 4 * j + 1] * wgt,
+                                   acc[16 * ch + 4 * j + 2] * wgt, acc[16 * ch + 4 * j + 3] * wgt);
+            *reinterpret_cast<float4*>(sw + lane * kStgStride + 4 * j) = v;
+          }
+          __syncwarp();
+#pragma unroll
+          for (int r4 = 0; r4 < 4; ++r4) {
+            const int rr = r4 * 8 + (lane >> 2);
+            const int cc = (lane & 3) * 4;
+            const int gg = __shfl_sync(0xffffffffu, g, rr);
+            const float4 v = *reinterpret_cast<const float4*>(sw + rr * kStgStride + cc);
+            if (gg >= 0)
+              red_add_v4(p.acc + static_cast<size_t>(gg) * p.H + col0 + 16 * ch + cc, v.x, v.y,
+                         v.z, v.w);
+          }
+          __syncwarp();
+        }
+        __threadfence();
+        __syncwarp();
+        bool last = false;
+        if (g >= 0) {
+          const int old = atomicAdd(&p.cnt[static_cast<size_t>(g) * p.n_tiles + c.nt], 1);
+          last = (old == 2 * p.tok_need[g] - 1);
+        }
+        unsigned lm = __ballot_sync(0xffffffffu, last);
+        while (lm) {
+          const int src = __ffs(lm) - 1;
+          lm &= lm - 1;
+          const int gg = __shfl_sync(0xffffffffu, g, src);
+          __threadfence();
+          float* rowp = p.acc + static_cast<size_t>(gg) * p.H + c.nt * kBN + lane * 8;
+          const float4 a = ld_cg_f4(rowp);
+          const float4 bq = ld_cg_f4(rowp + 4);
+          const int mt = p.tok_mt[gg];
+          const int m = mt >> 24, t = mt & 0xFFFFFF;
+          uint4 o;
+          o.x = pack_bf16x2(a.x, a.y);
+          o.y = pack_bf16x2(a.z, a.w);
+          o.z = pack_bf16x2(bq.x, bq.y);
+          o.w = pack_bf16x2(bq.z, bq.w);
+          *reinterpret_cast<uint4*>(ytab.y[m] + static_cast<size_t>(t) * p.H + c.nt * kBN +
+                                    lane * 8) = o;
+          __stcg(reinterpret_cast<float4*>(rowp), make_float4(0.f, 0.f, 0.f, 0.f));
+          __stcg(reinterpret_cast<float4*>(rowp + 4), make_float4(0.f, 0.f, 0.f, 0.f));
+          if (lane == 0) p.cnt[static_cast<size_t>(gg) * p.n_tiles + c.nt] = 0;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+}  // namespace afd

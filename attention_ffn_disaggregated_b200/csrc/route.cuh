@@ -1,0 +1,320 @@
+// Routing of the FFN-pool expert layer: slab intake, per-expert histogram, exclusive
+// scan with the GEMM tile schedule, stable (token, slot)-ordered permutation, and the
+// gather of routed FP8 rows into expert order.
+//
+// The attention ranks publish FP8 tokens and top-K routing metadata into this GPU's
+// receive buffers (FastAFD, "Methodology / System Design", item 2); the FFN GPU groups the
+// routed rows by expert for its grouped GEMMs (item 3). The order inside an expert's group
+// is ascending (token, slot) with tokens numbered slab-major, which makes the result
+// deterministic and independent of how the work is split across CTAs.
+#pragma once
+
+#include "ptx.cuh"
+
+namespace afd {
+
+constexpr int kRouteThreads = 256;
+constexpr int kChunkTokens = 256;   // tokens per routing CTA (one per thread)
+constexpr int kRouteWarps = kRouteThreads / 32;
+constexpr int kTokensPerWarp = kChunkTokens / kRouteWarps;
+constexpr int kTileM = 128;
+
+struct SlabTable {
+  const uint8_t* x[AFD_MAX_SLABS];
+  const float* xs[AFD_MAX_SLABS];
+  const int32_t* ids[AFD_MAX_SLABS];
+  const float* w[AFD_MAX_SLABS];
+  __nv_bfloat16* y[AFD_MAX_SLABS];
+};
+
+struct RouteParams {
+  const int32_t* counts;  // device [M]
+  int M, cap, K, H, e0, El, Eg, S, G;
+  int num_chunks;
+  int rpad;               // row stride of the transposed scale arrays, >= max_rows + 128
+  int32_t* slab_base;     // [M+1]
+  int32_t* info;          // [0] T, [1] R, [2] m-tiles
+  int32_t* chunk_hist;    // [num_chunks][max(El,1)]
+  int32_t* chunk_off;     // [num_chunks][max(El,1)]
+  int32_t* group_count;   // [G]
+  int32_t* group_off;     // [G+1]
+  int32_t* mtile_off;     // [G+1]
+  int32_t* tok_mt;        // [Tmax] (slab << 24) | row
+  int32_t* tok_need;      // [Tmax] contributions this GPU adds to the token
+  int32_t* pos;           // [Tmax*K]
+  int32_t* row_token;     // [rpad]
+  int32_t* row_k;         // [rpad]
+  float* row_w;           // [rpad]
+  uint8_t* a_perm;        // [rpad][H]
+  float* sa_t;            // [H/128][rpad]
+  int* status;
+};
+
+// Slab-major prefix of the valid row counts, clamped to [0, cap].
+__device__ __forceinline__ void load_slab_base(const RouteParams& p, int32_t* s_base) {
+  if (threadIdx.x == 0) {
+    int run = 0;
+    bool bad = false;
+    for (int m = 0; m < p.M; ++m) {
+      s_base[m] = run;
+      int n = p.counts[m];
+      if (n < 0 || n > p.cap) {
+        bad = true;
+        n = n < 0 ? 0 : p.cap;
+      }
+      run += n;
+    }
+    s_base[p.M] = run;
+    if (bad) atomicOr(p.status, AFD_STATUS_BAD_COUNT);
+  }
+  __syncthreads();
+}
+
+__device__ __forceinline__ int find_slab(const int32_t* s_base, int M, int g) {
+  int lo = 0, hi = M - 1;           // largest m with s_base[m] <= g
+  while (lo < hi) {
+    int mid = (lo + hi + 1) >> 1;
+    if (s_base[mid] <= g) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+// Classify the K slots of one token. Returns a mask of the slots that are valid and
+// local; `le[k]` receives the local group of slot k. Sets *bad for ids that are neither
+// -1 nor in [0, E_g), and for ids repeated from an earlier slot.
+__device__ __forceinline__ uint32_t classify_token(const int32_t* ids, int K, int e0, int El,
+                                                   int Eg, int* le, bool* bad) {
+  uint32_t mask = 0;
+  for (int k = 0; k < K; ++k) {
+    const int id = ids[k];
+    le[k] = -1;
+    if (id == -1) continue;
+    if (id < 0 || id >= Eg) { *bad = true; continue; }
+    bool dup = false;
+    for (int j = 0; j < k; ++j) dup |= (ids[j] == id);
+    if (dup) { *bad = true; continue; }
+    if (id >= e0 && id < e0 + El) {
+      le[k] = id - e0;
+      mask |= 1u << k;
+    }
+  }
+  return mask;
+}
+
+// 1. per-chunk histogram of local groups; token bookkeeping.
+__global__ void __launch_bounds__(kRouteThreads) route_count_kernel(
+    const __grid_constant__ RouteParams p, const __grid_constant__ SlabTable slabs) {
+  __shared__ int32_t s_base[AFD_MAX_SLABS + 1];
+  __shared__ int32_t s_hist[AFD_MAX_GROUPS];
+  load_slab_base(p, s_base);
+  const int T = s_base[p.M];
+  if (blockIdx.x == 0) {
+    for (int m = threadIdx.x; m <= p.M; m += blockDim.x) p.slab_base[m] = s_base[m];
+    if (threadIdx.x == 0) p.info[0] = T;
+  }
+  for (int e = threadIdx.x; e < p.El; e += blockDim.x) s_hist[e] = 0;
+  __syncthreads();
+  const int g = blockIdx.x * kChunkTokens + threadIdx.x;
+  if (g < T) {
+    const int m = find_slab(s_base, p.M, g);
+    const int t = g - s_base[m];
+    int32_t ids[AFD_MAX_TOP_K];
+    int le[AFD_MAX_TOP_K];
+    const int32_t* src = slabs.ids[m] + static_cast<size_t>(t) * p.K;
+    for (int k = 0; k < p.K; ++k) ids[k] = src[k];
+    bool bad = false;
+    uint32_t mask = classify_token(ids, p.K, p.e0, p.El, p.Eg, le, &bad);
+    for (int k = 0; k < p.K; ++k)
+      if (mask >> k & 1u) atomicAdd(&s_hist[le[k]], 1);
+    p.tok_mt[g] = (m << 24) | t;
+    p.tok_need[g] = __popc(mask) + p.S;
+    if (bad) atomicOr(p.status, AFD_STATUS_BAD_ROUTING);
+  }
+  __syncthreads();
+  int32_t* out = p.chunk_hist + static_cast<size_t>(blockIdx.x) * max(p.El, 1);
+  for (int e = threadIdx.x; e < p.El; e += blockDim.x) out[e] = s_hist[e];
+}
+
+// Block-wide exclusive scan of one value per thread (blockDim.x == 1024).
+__device__ __forceinline__ int block_exclusive_scan(int v, int* s_warp, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) s_warp[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int w = lane < (blockDim.x >> 5) ? s_warp[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    s_warp[lane] = w;  // inclusive over warps
+  }
+  __syncthreads();
+  const int excl = x - v + (warp > 0 ? s_warp[warp - 1] : 0);
+  *total = s_warp[(blockDim.x >> 5) - 1];
+  __syncthreads();
+  return excl;
+}
+
+// 2. chunk offsets per group, group offsets (exclusive scan) and the m-tile schedule.
+__global__ void __launch_bounds__(1024) route_scan_kernel(const __grid_constant__ RouteParams p) {
+  __shared__ int s_warp[32];
+  const int T = p.info[0];
+  const int chunks = (T + kChunkTokens - 1) / kChunkTokens;
+  const int El1 = max(p.El, 1);
+  for (int e = threadIdx.x; e < p.El; e += blockDim.x) {
+    int run = 0;
+    for (int c = 0; c < chunks; ++c) {
+      const size_t i = static_cast<size_t>(c) * El1 + e;
+      const int h = p.chunk_hist[i];
+      p.chunk_off[i] = run;
+      run += h;
+    }
+    p.group_count[e] = run;
+  }
+  __syncthreads();
+  if (p.S && threadIdx.x == 0) p.group_count[p.El] = T;
+  __syncthreads();
+  int base_rows = 0, base_tiles = 0;
+  for (int g0 = 0; g0 < p.G; g0 += blockDim.x) {
+    const int g = g0 + threadIdx.x;
+    const int cnt = g < p.G ? p.group_count[g] : 0;
+    int tot_rows, tot_tiles;
+    const int ex_rows = block_exclusive_scan(cnt, s_warp, &tot_rows);
+    const int ex_tiles = block_exclusive_scan((cnt + kTileM - 1) / kTileM, s_warp, &tot_tiles);
+    if (g < p.G) {
+      p.group_off[g] = base_rows + ex_rows;
+      p.mtile_off[g] = base_tiles + ex_tiles;
+    }
+    base_rows += tot_rows;
+    base_tiles += tot_tiles;
+  }
+  if (threadIdx.x == 0) {
+    p.group_off[p.G] = base_rows;
+    p.mtile_off[p.G] = base_tiles;
+    p.info[1] = base_rows;
+    p.info[2] = base_tiles;
+  }
+}
+
+// 3. stable placement of every local (token, slot) pair and of the shared rows.
+// Dynamic shared memory: s_run [warps][El] + s_key [warps][32*K] int32.
+__global__ void __launch_bounds__(kRouteThreads) route_scatter_kernel(
+    const __grid_constant__ RouteParams p, const __grid_constant__ SlabTable slabs) {
+  extern __shared__ int32_t s_dyn[];
+  __shared__ int32_t s_base[AFD_MAX_SLABS + 1];
+  const int El1 = max(p.El, 1);
+  int32_t* s_run = s_dyn;                                   // [warps][El1]
+  int32_t* s_key = s_dyn + kRouteWarps * El1;               // [warps][32*K]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int m = threadIdx.x; m <= p.M; m += blockDim.x) s_base[m] = p.slab_base[m];
+  for (int i = threadIdx.x; i < kRouteWarps * El1; i += blockDim.x) s_run[i] = 0;
+  __syncthreads();
+  const int T = s_base[p.M];
+  const int K = p.K;
+  const int g = blockIdx.x * kChunkTokens + warp * kTokensPerWarp + lane;
+  int m = 0, t = 0;
+  int32_t* mykeys = s_key + warp * 32 * K;
+  if (g < T) {
+    m = find_slab(s_base, p.M, g);
+    t = g - s_base[m];
+    int32_t ids[AFD_MAX_TOP_K];
+    int le[AFD_MAX_TOP_K];
+    const int32_t* src = slabs.ids[m] + static_cast<size_t>(t) * K;
+    for (int k = 0; k < K; ++k) ids[k] = src[k];
+    bool bad = false;
+    classify_token(ids, K, p.e0, p.El, p.Eg, le, &bad);
+    for (int k = 0; k < K; ++k) {
+      mykeys[lane * K + k] = le[k];
+      if (le[k] >= 0) atomicAdd(&s_run[warp * El1 + le[k]], 1);
+    }
+  } else {
+    for (int k = 0; k < K; ++k) mykeys[lane * K + k] = -1;
+  }
+  __syncthreads();
+  // per-warp starting row of every group: group base + chunk base + earlier warps
+  const int32_t* coff = p.chunk_off + static_cast<size_t>(blockIdx.x) * El1;
+  for (int e = threadIdx.x; e < p.El; e += blockDim.x) {
+    int run = p.group_off[e] + coff[e];
+    for (int w = 0; w < kRouteWarps; ++w) {
+      const int v = s_run[w * El1 + e];
+      s_run[w * El1 + e] = run;
+      run += v;
+    }
+  }
+  __syncthreads();
+  // walk this warp's pairs in (token, slot) order, 32 at a time
+  const int gw0 = blockIdx.x * kChunkTokens + warp * kTokensPerWarp;
+  for (int r = 0; r < K; ++r) {
+    const int pidx = r * 32 + lane;             // pair index inside the warp
+    const int tl = pidx / K, k = pidx - tl * K;
+    const int key = mykeys[pidx];
+    const unsigned peers = __match_any_sync(0xffffffffu, key);
+    if (key >= 0) {
+      const int rank = __popc(peers & lanemask_lt());
+      const int row = s_run[warp * El1 + key] + rank;
+      const int gg = gw0 + tl;
+      const int mm = find_slab(s_base, p.M, gg);
+      const int tt = gg - s_base[mm];
+      p.pos[static_cast<size_t>(gg) * K + k] = row;
+      p.row_token[row] = gg;
+      p.row_k[row] = k;
+      p.row_w[row] = slabs.w[mm][static_cast<size_t>(tt) * K + k];
+    } else {
+      const int gg = gw0 + tl;
+      if (gg < T) p.pos[static_cast<size_t>(gg) * K + k] = -1;
+    }
+    __syncwarp();
+    if (key >= 0 && (31 - __clz(peers)) == static_cast<int>(lane))
+      s_run[warp * El1 + key] += __popc(peers);
+    __syncwarp();
+  }
+  if (g < T && p.S) {
+    const int row = p.group_off[p.El] + g;
+    p.row_token[row] = g;
+    p.row_k[row] = -1;
+    p.row_w[row] = 1.0f;
+  }
+  // tokens that receive nothing from this GPU get zeros (only possible without a shared
+  // expert); everything else is written by the down-projection's combine
+  if (!p.S) {
+    unsigned need0 = __ballot_sync(0xffffffffu, g < T && p.tok_need[g] == 0);
+    while (need0) {
+      const int src_lane = __ffs(need0) - 1;
+      need0 &= need0 - 1;
+      const int mm = __shfl_sync(0xffffffffu, m, src_lane);
+      const int tt = __shfl_sync(0xffffffffu, t, src_lane);
+      uint4* dst = reinterpret_cast<uint4*>(slabs.y[mm] + static_cast<size_t>(tt) * p.H);
+      for (int i = lane; i < p.H / 8; i += 32) dst[i] = make_uint4(0, 0, 0, 0);
+    }
+  }
+}
+
+// 4. copy routed rows (FP8 codes and their per-128 scales) into expert order.
+// One warp per row; scales are stored transposed ([H/128][rpad]) so that a GEMM tile
+// reads one block's scales for 32 consecutive rows with one coalesced load.
+__global__ void __launch_bounds__(kRouteThreads) gather_rows_kernel(
+    const __grid_constant__ RouteParams p, const __grid_constant__ SlabTable slabs) {
+  const int R = p.info[1];
+  const int lane = threadIdx.x & 31;
+  const int nwarps = (gridDim.x * blockDim.x) >> 5;
+  const int KB = p.H / AFD_QBLOCK;
+  for (int r = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; r < R; r += nwarps) {
+    const int g = p.row_token[r];
+    const int mt = p.tok_mt[g];
+    const int m = mt >> 24, t = mt & 0xFFFFFF;
+    const uint4* src = reinterpret_cast<const uint4*>(slabs.x[m] + static_cast<size_t>(t) * p.H);
+    uint4* dst = reinterpret_cast<uint4*>(p.a_perm + static_cast<size_t>(r) * p.H);
+    for (int i = lane; i < p.H / 16; i += 32) dst[i] = __ldg(src + i);
+    const float* ssrc = slabs.xs[m] + static_cast<size_t>(t) * KB;
+    for (int kb = lane; kb < KB; kb += 32) p.sa_t[static_cast<size_t>(kb) * p.rpad + r] = ssrc[kb];
+  }
+}
+
+}  // namespace afd

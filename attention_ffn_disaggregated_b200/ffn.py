@@ -1,0 +1,219 @@
+"""ctypes binding of the C ABI in include/afd_ffn.h (argument marshalling only).
+
+Every step of the layer runs in the CUDA library; this module never computes any part of
+it. PyTorch supplies device memory and streams. If the library is missing the import of
+`lib()` raises: there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from ctypes import POINTER, c_char_p, c_float, c_int32, c_int64, c_uint8, c_void_p
+from typing import Optional, Sequence
+
+import numpy as np
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libafd_ffn.so")
+
+AFD_OK = 0
+STATUS_NAMES = {0: "AFD_OK", 1: "AFD_ERR_INVALID_ARGUMENT", 2: "AFD_ERR_UNSUPPORTED",
+                3: "AFD_ERR_OUT_OF_MEMORY", 4: "AFD_ERR_CUDA", 5: "AFD_ERR_BAD_ROUTING",
+                6: "AFD_ERR_TIMEOUT"}
+STATUS_BAD_ROUTING, STATUS_TIMEOUT, STATUS_BAD_COUNT = 0x1, 0x2, 0x4
+KERNEL_NAMES = ["route_count", "route_scan", "route_scatter", "gather_rows", "gemm13_swiglu",
+                "gemm2_combine"]
+
+
+class Config(ctypes.Structure):
+    _fields_ = [("hidden", c_int32), ("intermediate", c_int32), ("num_experts_global", c_int32),
+                ("expert_begin", c_int32), ("num_local_experts", c_int32),
+                ("has_shared_expert", c_int32), ("top_k", c_int32), ("num_slabs", c_int32),
+                ("slab_capacity", c_int32)]
+
+
+class Weights(ctypes.Structure):
+    _fields_ = [("w13", c_void_p), ("w13_scale", c_void_p), ("w2", c_void_p), ("w2_scale", c_void_p)]
+
+
+class SlabDesc(ctypes.Structure):
+    _fields_ = [("x", c_void_p), ("x_scale", c_void_p), ("topk_ids", c_void_p),
+                ("topk_weights", c_void_p), ("y", c_void_p)]
+
+
+class PlanInfo(ctypes.Structure):
+    _fields_ = [("num_groups", c_int32), ("max_tokens", c_int32), ("max_rows", c_int32),
+                ("num_sms", c_int32), ("workspace_bytes", c_int64)]
+
+
+class AfdError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {STATUS_NAMES.get(code, code)}")
+        self.code = code
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libafd_ffn.so (built in-tree by build.py). Raises if it is missing."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"CUDA library not built: {LIB_PATH} (run attention_ffn_disaggregated_b200/build.py)")
+    L = ctypes.CDLL(LIB_PATH)
+    P = c_void_p
+    sig = {
+        "afd_ffn_check_config": (c_int32, [POINTER(Config)]),
+        "afd_ffn_plan": (c_int32, [POINTER(Config), POINTER(Weights), POINTER(c_void_p)]),
+        "afd_ffn_layer": (c_int32, [P, POINTER(SlabDesc), P, P]),
+        "afd_ffn_destroy": (None, [P]),
+        "afd_ffn_get_info": (c_int32, [P, POINTER(PlanInfo)]),
+        "afd_ffn_get_status": (c_int32, [P, P, POINTER(c_int32)]),
+        "afd_ffn_read_routing": (c_int32, [P, P, POINTER(c_int32), POINTER(c_int32), P, P, P, P, P, P]),
+        "afd_ffn_read_intermediate": (c_int32, [P, P, P, P]),
+        "afd_ffn_set_timing": (c_int32, [P, c_int32]),
+        "afd_ffn_get_kernel_times": (c_int32, [P, POINTER(c_float)]),
+        "afd_ffn_set_wait_limit": (c_int32, [P, c_int64]),
+        "afd_ffn_inject_stall": (c_int32, [P, c_int32]),
+        "afd_ffn_kernels_per_layer": (c_int32, []),
+        "afd_status_string": (c_char_p, [c_int32]),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(L, name)
+        f.restype = res
+        f.argtypes = args
+    _lib = L
+    return L
+
+
+def make_config(shape, num_slabs: int, slab_capacity: int) -> Config:
+    return Config(shape.hidden, shape.intermediate, shape.num_experts_global, shape.expert_begin,
+                  shape.num_local_experts, shape.has_shared_expert, shape.top_k, num_slabs,
+                  slab_capacity)
+
+
+def check_config(cfg: Config) -> int:
+    return lib().afd_ffn_check_config(ctypes.byref(cfg))
+
+
+def _ptr(t) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream_handle(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        stream = torch.cuda.current_stream()
+    h = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+    return h or None
+
+
+class FfnLayer:
+    """One FFN-pool expert layer on the current CUDA device.
+
+    w13/w13_scale/w2/w2_scale: CUDA tensors in the layouts of include/afd_ffn.h (uint8 codes,
+    float32 scales); they are kept referenced for the plan's lifetime.
+    """
+
+    def __init__(self, shape, num_slabs: int, slab_capacity: int, w13, w13_scale, w2, w2_scale):
+        L = lib()
+        self.shape = shape
+        self.num_slabs = num_slabs
+        self.slab_capacity = slab_capacity
+        self._keep = (w13, w13_scale, w2, w2_scale)
+        self.cfg = make_config(shape, num_slabs, slab_capacity)
+        w = Weights(_ptr(w13), _ptr(w13_scale), _ptr(w2), _ptr(w2_scale))
+        h = c_void_p()
+        rc = L.afd_ffn_plan(ctypes.byref(self.cfg), ctypes.byref(w), ctypes.byref(h))
+        if rc != AFD_OK:
+            raise AfdError(rc, "afd_ffn_plan")
+        self.plan = h
+        self.info = PlanInfo()
+        L.afd_ffn_get_info(self.plan, ctypes.byref(self.info))
+        self._descs = (SlabDesc * num_slabs)()
+
+    def close(self):
+        if getattr(self, "plan", None):
+            lib().afd_ffn_destroy(self.plan)
+            self.plan = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def __call__(self, slabs: Sequence, counts, stream=None) -> None:
+        """slabs: sequence of objects with .x .x_scale .topk_ids .topk_weights .y CUDA tensors."""
+        if len(slabs) != self.num_slabs:
+            raise ValueError("expected %d slabs" % self.num_slabs)
+        for i, s in enumerate(slabs):
+            self._descs[i] = SlabDesc(_ptr(s.x), _ptr(s.x_scale), _ptr(s.topk_ids),
+                                      _ptr(s.topk_weights), _ptr(s.y))
+        rc = lib().afd_ffn_layer(self.plan, self._descs, c_void_p(_ptr(counts)),
+                                 c_void_p(_stream_handle(stream)))
+        if rc != AFD_OK:
+            raise AfdError(rc, "afd_ffn_layer")
+
+    def status(self, stream=None):
+        word = c_int32(0)
+        rc = lib().afd_ffn_get_status(self.plan, c_void_p(_stream_handle(stream)), ctypes.byref(word))
+        return rc, word.value
+
+    def routing(self, stream=None) -> dict:
+        inf = self.info
+        G, R, T = inf.num_groups, inf.max_rows, inf.max_tokens
+        K = self.shape.top_k
+        nt, nr = c_int32(0), c_int32(0)
+        counts = np.zeros(G, np.int32)
+        offsets = np.zeros(G + 1, np.int32)
+        row_token = np.zeros(max(R, 1), np.int32)
+        row_k = np.zeros(max(R, 1), np.int32)
+        row_w = np.zeros(max(R, 1), np.float32)
+        pos = np.zeros(max(T * K, 1), np.int32)
+        rc = lib().afd_ffn_read_routing(
+            self.plan, c_void_p(_stream_handle(stream)), ctypes.byref(nt), ctypes.byref(nr),
+            counts.ctypes.data, offsets.ctypes.data, row_token.ctypes.data, row_k.ctypes.data,
+            row_w.ctypes.data, pos.ctypes.data)
+        if rc != AFD_OK:
+            raise AfdError(rc, "afd_ffn_read_routing")
+        r = nr.value
+        return {"num_tokens": nt.value, "num_rows": r, "counts": counts, "offsets": offsets,
+                "row_token": row_token[:r], "row_k": row_k[:r], "row_weight": row_w[:r],
+                "pos": pos[:nt.value * K]}
+
+    def intermediate(self, stream=None):
+        R = self.info.max_rows
+        I = self.shape.intermediate
+        codes = np.zeros((max(R, 1), I), np.uint8)
+        scales = np.zeros((max(R, 1), I // 128), np.float32)
+        rc = lib().afd_ffn_read_intermediate(self.plan, c_void_p(_stream_handle(stream)),
+                                             codes.ctypes.data, scales.ctypes.data)
+        if rc != AFD_OK:
+            raise AfdError(rc, "afd_ffn_read_intermediate")
+        n = self.routing(stream)["num_rows"]
+        return codes[:n], scales[:n]
+
+    def set_timing(self, enable: bool):
+        lib().afd_ffn_set_timing(self.plan, 1 if enable else 0)
+
+    def kernel_times(self):
+        ms = (c_float * len(KERNEL_NAMES))()
+        rc = lib().afd_ffn_get_kernel_times(self.plan, ms)
+        if rc != AFD_OK:
+            raise AfdError(rc, "afd_ffn_get_kernel_times")
+        return dict(zip(KERNEL_NAMES, list(ms)))
+
+    def set_wait_limit(self, ns: int):
+        rc = lib().afd_ffn_set_wait_limit(self.plan, int(ns))
+        if rc != AFD_OK:
+            raise AfdError(rc, "afd_ffn_set_wait_limit")
+
+    def inject_stall(self, enable: bool = True):
+        lib().afd_ffn_inject_stall(self.plan, 1 if enable else 0)
+
+
+def kernels_per_layer() -> int:
+    return lib().afd_ffn_kernels_per_layer()

@@ -1,0 +1,385 @@
+#!/usr/bin/env python3
+"""Benchmark of the FFN-pool expert layer (one step = one full layer call: routing,
+W13 + SwiGLU, W2 + top-K combine) on synthetic inputs shaped like the pages' models.
+
+Default workload: the DeepSeek-V3-shaped FFN-pool share (H 7168, I 2048, 32 of 256 routed
+experts held here plus 1 shared expert, top-8, 4096 tokens over 16 slabs, Zipf s=1
+popularity). One JSON line on stdout (rank 0).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
+
+Multi-GPU (torchrun, one process per GPU): every rank is an independent FFN replica with
+its own batch (data-parallel FFN pools over disjoint slab sets need no exchange), so the
+scaling is weak and value = all ranks' tokens / max over ranks of the device time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "MoE FFN-layer routed tokens/s at 1 B200; % of HBM / FP8 tensor roofline"
+DEFAULT_CONFIG = "deepseek_v3_share_t4096"
+FLUSH_BYTES = 256 << 20
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default=DEFAULT_CONFIG)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-sample-tokens", type=int, default=64)
+    return ap.parse_args()
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", 0)), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def workload_bytes_flops(inp, routing_counts):
+    """Algorithmic bytes and FLOPs of one layer call.
+
+    bytes = weights (codes + scales) of experts that receive rows + x codes + x scales
+            + ids and weights + bf16 output;  FLOPs = 6 * H * I * R.
+    """
+    sh = inp.shape
+    H, I, K = sh.hidden, sh.intermediate, sh.top_k
+    T = int(np.sum(inp.counts))
+    active = int(np.count_nonzero(routing_counts))
+    w_bytes_per_expert = 3 * H * I + (2 * I // 128) * (H // 128) * 4 + (H // 128) * (I // 128) * 4
+    R = int(np.sum(routing_counts))
+    bytes_ = active * w_bytes_per_expert + T * H + T * (H // 128) * 4 + T * K * 8 + T * H * 2
+    flops = 6.0 * H * I * R
+    return bytes_, flops, R, active
+
+
+def source_hash():
+    h = hashlib.sha256()
+    for d in ("attention_ffn_disaggregated_b200/csrc", "include"):
+        for f in sorted(os.listdir(os.path.join(ROOT, d))):
+            h.update(open(os.path.join(ROOT, d, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel: str):
+    """DRAM bytes per launch recorded by ncu for this kernel source (None if stale/missing)."""
+    p = os.path.join(ROOT, "profiles", f"{kernel}_traffic.txt")
+    if not os.path.exists(p):
+        return None
+    kv = {}
+    for line in open(p):
+        if ":" in line and not line.startswith("#"):
+            k, v = line.split(":", 1)
+            kv[k.strip()] = v.strip()
+    if kv.get("source_sha") != source_hash():
+        return None
+    try:
+        return float(kv["dram_bytes_per_launch_full"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"afd_clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if not self.proc or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        sms, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sms.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sms:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": ["no samples"]}
+        loaded = [s for s in sms if s > 0.5 * (mx or 1)] or sms
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sms)}
+
+
+def cpu_baseline(inp, n_tokens):
+    """The oracle as it stands, on the host cores, on a bounded token sample."""
+    from oracle import ffn as offn
+    T = int(np.sum(inp.counts))
+    toks = np.linspace(0, T - 1, num=min(n_tokens, T)).astype(np.int64)
+    rt = offn.route_inputs(inp)
+    t0 = time.perf_counter()
+    offn.ffn_layer(inp, tokens=toks, routing=rt)
+    dt = time.perf_counter() - t0
+    cores = os.cpu_count()
+    try:
+        from threadpoolctl import threadpool_info
+        nt = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        if nt:
+            cores = int(max(nt))
+    except Exception:
+        pass
+    return {"value": len(toks) / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{len(toks)} of {T} tokens (evenly spaced), full routing, float64 dequantise "
+                      f"+ grouped SwiGLU FFN + requant + combine; {dt:.1f} s"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    wl = W.workload_by_name(args.config)
+    inp = W.make_inputs(wl)
+    from oracle import ffn as offn
+    T = int(np.sum(inp.counts))
+    per_step = max(1, min(T, 8))
+    rt = offn.route_inputs(inp)
+    times = []
+    for i in range(args.warmup + args.steps):
+        toks = (np.arange(per_step) * 97 + i * 13) % T
+        t0 = time.perf_counter()
+        offn.ffn_layer(inp, tokens=toks, routing=rt)
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    tot = sum(times)
+    value = per_step * len(times) / tot
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * tot / len(times), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "tokens": T, "slabs": wl.num_slabs},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": os.cpu_count(), "kind": "oracle",
+                         "sample": f"{per_step} tokens per step of the {T}-token workload"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+    from attention_ffn_disaggregated_b200 import FfnLayer, kernels_per_layer
+    from attention_ffn_disaggregated_b200.device import (to_device_counts, to_device_slabs,
+                                                          to_device_weights)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    base = W.workload_by_name(args.config)
+    wl = W.Workload(base.name, base.shape, base.num_tokens, base.num_slabs, base.zipf_s,
+                    base.zero_pop_mod, seed=tuple(base.seed) if rank == 0 else (base.seed[0], 1000 + rank))
+    weights = None
+    if rank != 0:
+        weights = W.make_weights(wl.shape, __import__("torch").Generator().manual_seed(
+            int(np.random.SeedSequence(list(base.seed)).generate_state(1)[0])))
+    inp = W.make_inputs(wl, weights=weights)
+    T = int(np.sum(inp.counts))
+    dev_w = to_device_weights(inp)
+    layer = FfnLayer(inp.shape, len(inp.slabs), inp.capacity, *dev_w)
+    slabs = to_device_slabs(inp, y_fill=0.0)
+    counts = to_device_counts(inp)
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    layer(slabs, counts)
+    rc, word = layer.status()
+    if rc != 0:
+        raise RuntimeError(f"layer status {rc} word {word:#x}")
+    rt = layer.routing()
+    bytes_alg, flops_alg, R, active = workload_bytes_flops(inp, rt["counts"])
+
+    layer.set_timing(True)
+    for _ in range(args.warmup):
+        flush.zero_()
+        layer(slabs, counts)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+
+    kt = {k: [] for k in ("route_count", "route_scan", "route_scatter", "gather_rows",
+                          "gemm13_swiglu", "gemm2_combine")}
+    step_ms = []
+    with ClockSampler(local) as clk:
+        for _ in range(args.steps):
+            flush.zero_()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            layer(slabs, counts)
+            e1.record(stream)
+            e1.synchronize()
+            step_ms.append(e0.elapsed_time(e1))
+            for k, v in layer.kernel_times().items():
+                kt[k].append(v)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    tot_ms = float(sum(step_ms))
+    if world > 1:
+        t = torch.tensor([tot_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        tot_ms = float(t.item())
+    rc, word = layer.status()
+    if rc != 0:
+        raise RuntimeError(f"layer status {rc} word {word:#x} after timing")
+
+    # end to end through the C ABI with host buffers: pinned H2D of the step's inputs,
+    # the layer, D2H of the outputs, all inside the timed region
+    layer.set_timing(False)
+    host = []
+    h2d = 0
+    for s in slabs:
+        hs = {n: getattr(s, n).cpu().pin_memory() for n in ("x", "x_scale", "topk_ids", "topk_weights")}
+        host.append(hs)
+        h2d += sum(v.numel() * v.element_size() for v in hs.values())
+    counts_h = counts.cpu().pin_memory()
+    h2d += counts_h.numel() * 4
+    y_h = [torch.empty_like(s.y, device="cpu").pin_memory() for s in slabs]
+    d2h = sum(int(n) * inp.shape.hidden * 2 for n in inp.counts)
+    e2e_ms = []
+    for i in range(args.warmup + args.steps):
+        flush.zero_()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for s, hs in zip(slabs, host):
+            for n, v in hs.items():
+                getattr(s, n).copy_(v, non_blocking=True)
+        counts.copy_(counts_h, non_blocking=True)
+        layer(slabs, counts)
+        for s, yh, n in zip(slabs, y_h, inp.counts):
+            yh[:int(n)].copy_(s.y[:int(n)], non_blocking=True)
+        e1.record(stream)
+        e1.synchronize()
+        if i >= args.warmup:
+            e2e_ms.append(e0.elapsed_time(e1))
+    e2e_tot = float(sum(e2e_ms))
+    if world > 1:
+        t = torch.tensor([e2e_tot], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_tot = float(t.item())
+
+    hbm, bf16, bf16_sus, peak_src = measured_peaks()
+    fp8_peak = 2.0 * bf16          # measured bf16 burst x nominal fp8/bf16 ratio 2
+    mean = {k: float(np.mean(v)) for k, v in kt.items()}
+    dominant = max(("gemm13_swiglu", "gemm2_combine"), key=lambda k: mean[k])
+    H, I = inp.shape.hidden, inp.shape.intermediate
+    flops_k = (4.0 if dominant == "gemm13_swiglu" else 2.0) * H * I * R
+    achieved = flops_k / (mean[dominant] * 1e-3) / 1e12
+    t_roof = max(bytes_alg / (hbm * 1e9), flops_alg / (fp8_peak * 1e12))
+    layer_ms = tot_ms / args.steps
+    bound = "tensor" if flops_alg / (fp8_peak * 1e12) >= bytes_alg / (hbm * 1e9) else "hbm"
+
+    if rank == 0:
+        cpu = None
+        if not args.no_cpu_baseline and world == 1:
+            cpu = cpu_baseline(inp, args.cpu_sample_tokens)
+        line = {
+            "metric": METRIC,
+            "value": world * args.steps * T / (tot_ms * 1e-3),
+            "unit": "tokens/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": layer_ms,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "fp8_e4m3",
+            "data": "synthetic",
+            "config": {"workload": wl.name, "tokens": T, "slabs": wl.num_slabs, "hidden": H,
+                       "intermediate": I, "local_experts": inp.shape.num_local_experts,
+                       "shared_expert": inp.shape.has_shared_expert, "top_k": inp.shape.top_k,
+                       "routed_rows": R, "active_experts": active,
+                       "l2": "flushed between steps (256 MiB write, untimed)",
+                       "parallelism": f"replica x{world}"},
+            "roofline": {"bound": "tensor", "kernel": dominant, "achieved": achieved,
+                         "peak": fp8_peak, "unit": "TFLOP/s", "frac": achieved / fp8_peak,
+                         "traffic": profiled_traffic(dominant),
+                         "peak_source": f"{peak_src} bf16 burst x 2 (fp8/bf16 nominal ratio)"},
+            "layer_roofline": {"bound": bound, "t_roof_ms": t_roof * 1e3, "t_layer_ms": layer_ms,
+                               "frac": t_roof * 1e3 / layer_ms, "alg_bytes": bytes_alg,
+                               "alg_flops": flops_alg, "hbm_gbs": hbm, "fp8_tflops": fp8_peak},
+            "kernel_ms": mean,
+            "routed_rows_per_s": world * args.steps * R / (tot_ms * 1e-3),
+            "e2e": {"value": world * args.steps * T / (e2e_tot * 1e-3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": kernels_per_layer() * args.steps,
+            "clocks": clk.summary(),
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    del layer
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,224 @@
+/*
+ * afd_ffn.h -- C ABI of the FFN-pool expert layer of attention-FFN disaggregation (AFD).
+ *
+ * What the layer computes (FastAFD, "Methodology / System Design", items 1-3; vLLM AFD
+ * plugin, "FFN service"): M attention ranks have published block-FP8 token activations
+ * and their top-K routing (expert ids and combine weights) into M receive buffers
+ * ("slabs") on this GPU. For every token the layer evaluates each routed expert that
+ * this GPU holds, plus an optional shared expert, as
+ *
+ *     G = x . W13^T (block-FP8),  h = silu(G[:I]) * G[I:],  h -> e4m3 per (row, 128),
+ *     Y = h . W2^T  (block-FP8),
+ *
+ * and writes  y = sum_k w_k * Y_k  (+ Y_shared)  as bf16 into the token's row of its slab.
+ * Routing ids outside [expert_begin, expert_begin + num_local_experts) belong to other
+ * FFN GPUs and are skipped, so y is this GPU's partial sum.
+ *
+ * Data formats (all device memory, row-major, caller-owned):
+ *   e4m3      OCP FP8 E4M3 "fn" codes, one byte per element.
+ *   W13       e4m3 [E][2I][H]: rows 0..I-1 are the gate projection, rows I..2I-1 the up
+ *             projection. Scale fp32 [E][2I/128][H/128], one per 128x128 block.
+ *   W2        e4m3 [E][H][I]. Scale fp32 [E][H/128][I/128].
+ *             E = num_local_experts + has_shared_expert; the shared expert is index
+ *             num_local_experts. Routing id i maps to weight index i - expert_begin.
+ *   slab m    x e4m3 [cap][H], x_scale fp32 [cap][H/128] (one scale per token per 128
+ *             channels), topk_ids int32 [cap][K] (global expert ids, -1 = empty slot),
+ *             topk_weights fp32 [cap][K], y bf16 [cap][H] (output; rows < n_m written).
+ *   counts    device int32 [M]: n_m, the number of valid rows of slab m (0 <= n_m <= cap).
+ *
+ * Routing rules: slot k of token t is used iff its id is in [0, E_g), not equal to an id
+ * in an earlier slot of the same token, and local. An id that is neither -1 nor in
+ * [0, E_g), or a repeated id, is skipped and sets AFD_STATUS_BAD_ROUTING in the plan's
+ * device status word. Routed rows are grouped by expert in ascending (token, slot) order
+ * with tokens numbered slab-major; this order is deterministic.
+ *
+ * Errors: functions return afd_status_t. Argument errors return before anything is
+ * enqueued. Conditions detected on the device (bad routing ids, slab counts above the
+ * capacity, a bounded wait that expired) are OR-ed into the plan's status word, read
+ * with afd_ffn_get_status(); the kernels never trap.
+ *
+ * Threading: a plan is not thread-safe; calls on one plan must be serialised by the
+ * caller, and layer calls on one plan must be ordered on the GPU (one stream, or
+ * explicit events) because they share the plan's workspace.
+ */
+#ifndef AFD_FFN_H_
+#define AFD_FFN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define AFD_API __attribute__((visibility("default")))
+#else
+#define AFD_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  AFD_OK = 0,
+  AFD_ERR_INVALID_ARGUMENT = 1, /* bad pointer, size or shape; nothing was enqueued */
+  AFD_ERR_UNSUPPORTED = 2,      /* no sm_100 device, or a shape outside the supported limits */
+  AFD_ERR_OUT_OF_MEMORY = 3,    /* workspace allocation failed */
+  AFD_ERR_CUDA = 4,             /* a CUDA runtime call or launch failed */
+  AFD_ERR_BAD_ROUTING = 5,      /* returned by afd_ffn_get_status when the device saw bad ids */
+  AFD_ERR_TIMEOUT = 6           /* returned by afd_ffn_get_status when a device wait expired */
+} afd_status_t;
+
+/* Bits of the device status word. */
+#define AFD_STATUS_BAD_ROUTING 0x1 /* id outside [0, E_g) and != -1, or repeated in a token */
+#define AFD_STATUS_TIMEOUT 0x2     /* a bounded device wait expired; outputs are invalid */
+#define AFD_STATUS_BAD_COUNT 0x4   /* some counts[m] < 0 or > slab_capacity; clamped */
+
+/* Limits. */
+#define AFD_MAX_SLABS 128
+#define AFD_MAX_TOP_K 32
+#define AFD_MAX_GROUPS 1024 /* num_local_experts + has_shared_expert */
+#define AFD_QBLOCK 128      /* quantisation block edge */
+
+/* Device kernels of one layer call, in launch order (for afd_ffn_get_kernel_times). */
+#define AFD_KERNEL_ROUTE_COUNT 0
+#define AFD_KERNEL_ROUTE_SCAN 1
+#define AFD_KERNEL_ROUTE_SCATTER 2
+#define AFD_KERNEL_GATHER 3
+#define AFD_KERNEL_GEMM13 4
+#define AFD_KERNEL_GEMM2 5
+#define AFD_NUM_KERNELS 6
+
+struct CUstream_st;
+typedef struct CUstream_st* afd_stream_t; /* same type as cudaStream_t; NULL = legacy stream */
+
+typedef struct afd_ffn_plan_s* afd_ffn_plan_t; /* opaque; owned by the library */
+
+typedef struct {
+  int32_t hidden;             /* H, multiple of 128 */
+  int32_t intermediate;       /* I, multiple of 128 */
+  int32_t num_experts_global; /* E_g >= 1: ids the router may emit are [0, E_g) */
+  int32_t expert_begin;       /* e0 >= 0 */
+  int32_t num_local_experts;  /* E_l >= 0, e0 + E_l <= E_g */
+  int32_t has_shared_expert;  /* S in {0, 1}; E_l + S >= 1 */
+  int32_t top_k;              /* K in [1, min(E_g, AFD_MAX_TOP_K)] */
+  int32_t num_slabs;          /* M in [1, AFD_MAX_SLABS] */
+  int32_t slab_capacity;      /* cap >= 1: rows allocated per slab */
+} afd_ffn_config_t;
+
+typedef struct {
+  const void* w13;        /* e4m3 [E][2I][H], 16-byte aligned */
+  const float* w13_scale; /* fp32 [E][2I/128][H/128] */
+  const void* w2;         /* e4m3 [E][H][I], 16-byte aligned */
+  const float* w2_scale;  /* fp32 [E][H/128][I/128] */
+} afd_ffn_weights_t;
+
+typedef struct {
+  const void* x;              /* e4m3 [cap][H], 16-byte aligned */
+  const float* x_scale;       /* fp32 [cap][H/128] */
+  const int32_t* topk_ids;    /* int32 [cap][K] */
+  const float* topk_weights;  /* fp32 [cap][K] */
+  void* y;                    /* bf16 [cap][H], 16-byte aligned; rows < n_m are written */
+} afd_slab_t;
+
+/* Host-visible sizes of a plan (for sizing inspection buffers). */
+typedef struct {
+  int32_t num_groups;     /* G = E_l + S */
+  int32_t max_tokens;     /* M * cap */
+  int32_t max_rows;       /* M * cap * (min(K, E_l) + S): routed rows the workspace holds */
+  int32_t num_sms;        /* grid of the persistent GEMM kernels */
+  int64_t workspace_bytes;
+} afd_ffn_plan_info_t;
+
+/*
+ * Validate a configuration without touching the GPU. AFD_OK or
+ * AFD_ERR_INVALID_ARGUMENT (cfg NULL or a field out of range) or AFD_ERR_UNSUPPORTED
+ * (a limit above is exceeded).
+ */
+AFD_API afd_status_t afd_ffn_check_config(const afd_ffn_config_t* cfg);
+
+/*
+ * Build a plan for one layer on the current CUDA device: validates cfg and weights,
+ * checks for an sm_100 device, allocates the workspace (cudaMalloc; freed by
+ * afd_ffn_destroy), zeroes the combine accumulators and encodes the TMA descriptors of
+ * the weights. The weights are read by every later layer call and must stay valid and
+ * unchanged until afd_ffn_destroy. Synchronous. On error *out is set to NULL.
+ */
+AFD_API afd_status_t afd_ffn_plan(const afd_ffn_config_t* cfg, const afd_ffn_weights_t* weights,
+                          afd_ffn_plan_t* out);
+
+/*
+ * Enqueue one layer evaluation on `stream`; never synchronises with the host.
+ * slabs: host array of num_slabs descriptors (read during the call only; the device
+ * buffers they point to must stay valid until the stream reaches the work).
+ * d_counts: device int32 [num_slabs]. Returns AFD_ERR_INVALID_ARGUMENT for NULL
+ * arguments or misaligned slab pointers (nothing enqueued) and AFD_ERR_CUDA if a
+ * launch fails.
+ */
+AFD_API afd_status_t afd_ffn_layer(afd_ffn_plan_t plan, const afd_slab_t* slabs, const int32_t* d_counts,
+                           afd_stream_t stream);
+
+/* Free the plan and its workspace. NULL is a no-op. Synchronises the device. */
+AFD_API void afd_ffn_destroy(afd_ffn_plan_t plan);
+
+/* Sizes of a plan. */
+AFD_API afd_status_t afd_ffn_get_info(afd_ffn_plan_t plan, afd_ffn_plan_info_t* info);
+
+/*
+ * Synchronise `stream`, read the device status word into *status_word (may be NULL),
+ * and clear it. Returns AFD_ERR_TIMEOUT if the TIMEOUT bit was set, else
+ * AFD_ERR_BAD_ROUTING if BAD_ROUTING or BAD_COUNT was set, else AFD_OK.
+ */
+AFD_API afd_status_t afd_ffn_get_status(afd_ffn_plan_t plan, afd_stream_t stream, int32_t* status_word);
+
+/*
+ * Copy the routing of the last layer call to HOST buffers after synchronising `stream`.
+ * Any pointer may be NULL to skip that array. Sizes: counts [G], offsets [G+1],
+ * row_token / row_k / row_weight [max_rows] (first num_rows valid), pos [max_tokens*K]
+ * (first num_tokens*K valid). row_k is -1 for shared-expert rows; pos is -1 for slots
+ * that are not local.
+ */
+AFD_API afd_status_t afd_ffn_read_routing(afd_ffn_plan_t plan, afd_stream_t stream, int32_t* num_tokens,
+                                  int32_t* num_rows, int32_t* counts, int32_t* offsets,
+                                  int32_t* row_token, int32_t* row_k, float* row_weight,
+                                  int32_t* pos);
+
+/*
+ * Copy the intermediate of the last layer call to HOST buffers after synchronising
+ * `stream`: h_codes e4m3 [max_rows][I] and h_scales fp32 [max_rows][I/128]
+ * (first num_rows rows valid). Either pointer may be NULL.
+ */
+AFD_API afd_status_t afd_ffn_read_intermediate(afd_ffn_plan_t plan, afd_stream_t stream,
+                                       uint8_t* h_codes, float* h_scales);
+
+/*
+ * Per-kernel timing. When enabled, layer calls record CUDA events around each kernel
+ * on the launch stream. afd_ffn_get_kernel_times waits for the last call's events and
+ * writes AFD_NUM_KERNELS durations in milliseconds (index = AFD_KERNEL_*).
+ */
+AFD_API afd_status_t afd_ffn_set_timing(afd_ffn_plan_t plan, int32_t enable);
+AFD_API afd_status_t afd_ffn_get_kernel_times(afd_ffn_plan_t plan, float* ms);
+
+/*
+ * Limit, in nanoseconds, of every bounded device wait (default 1e9). Used by tests to
+ * make an injected stall expire quickly.
+ */
+AFD_API afd_status_t afd_ffn_set_wait_limit(afd_ffn_plan_t plan, int64_t limit_ns);
+
+/*
+ * Test hook: when `enable` is non-zero, the next layer call's W13 producer skips one
+ * stage so that the consumer's bounded wait expires and sets AFD_STATUS_TIMEOUT.
+ * The layer's outputs are then invalid. Host-side fault injection only; it does not
+ * fault the GPU.
+ */
+AFD_API afd_status_t afd_ffn_inject_stall(afd_ffn_plan_t plan, int32_t enable);
+
+/* Number of this library's kernels one afd_ffn_layer call launches. */
+AFD_API int32_t afd_ffn_kernels_per_layer(void);
+
+/* Human-readable name of a status code. */
+AFD_API const char* afd_status_string(afd_status_t s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* AFD_FFN_H_ */

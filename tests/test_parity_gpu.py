@@ -1,0 +1,150 @@
+"""GPU parity: the CUDA layer (through the C ABI) against the CPU oracle.
+
+Routing arrays (counts, offsets, row order, slots, weights, pos) must be bit-exact. Each
+bf16 output row must satisfy max|gpu - oracle| <= 2e-2 x RMS(oracle row); rows with no
+contribution must be exactly zero. Sizes here span several 128-row and 256-column tiles
+with ragged tails; the full-size workloads are checked on sampled tokens.
+"""
+import numpy as np
+import pytest
+
+import workloads as W
+from oracle import ffn as offn
+from tests.helpers import compare_outputs, compare_routing, run_cuda_layer
+
+pytestmark = pytest.mark.gpu
+
+
+def _full_check(inp, calls=1):
+    res = run_cuda_layer(inp, calls=calls)
+    ref = offn.ffn_layer(inp)
+    compare_routing(res["routing"], ref["routing"])
+    worst = [compare_outputs(o, ref["out"]) for o in res["outs"]]
+    return res, ref, worst
+
+
+def test_tiny_config():
+    inp = W.make_inputs(W.CONFIGS["tiny"])
+    res, ref, _ = _full_check(inp)
+    assert res["status_rc"] == 0
+
+
+@pytest.mark.parametrize("seed,shape,counts,cap,zipf", [
+    (1, W.LayerShape(512, 256, 16, 0, 16, 0, 4), [300, 0, 177, 41], 300, None),
+    (2, W.LayerShape(768, 384, 24, 8, 10, 1, 6), [129, 255, 1], 256, 1.0),
+    (3, W.LayerShape(1024, 512, 8, 0, 8, 1, 2), [1000], 1000, 0.5),
+    (4, W.LayerShape(256, 128, 64, 0, 64, 0, 8), [513, 77, 0, 3, 250], 513, 1.2),
+])
+def test_random_shapes_several_tiles(seed, shape, counts, cap, zipf):
+    inp = W.make_custom_inputs(shape, counts, cap, seed=seed, zipf_s=zipf)
+    res, _, _ = _full_check(inp)
+    assert res["status_rc"] == 0
+
+
+def test_repeated_calls_self_clean():
+    """The combine accumulators are cleared by the last contributor: call twice, same result."""
+    inp = W.make_custom_inputs(W.LayerShape(512, 256, 12, 2, 8, 1, 4), [200, 90], 200, seed=7)
+    res, ref, worst = _full_check(inp, calls=3)
+    assert len(worst) == 3
+
+
+def test_empty_batch_and_empty_slabs():
+    sh = W.LayerShape(256, 128, 8, 0, 8, 1, 2)
+    inp = W.make_custom_inputs(sh, [0, 0, 0], 4, seed=8)
+    res = run_cuda_layer(inp)
+    assert res["routing"]["num_tokens"] == 0 and res["routing"]["num_rows"] == 0
+    assert res["status_rc"] == 0
+    inp = W.make_custom_inputs(sh, [0, 1, 0], 4, seed=9)
+    _full_check(inp)
+
+
+def test_no_local_contribution_rows_are_zero():
+    """Without a shared expert, tokens whose ids are all non-local get exact zeros."""
+    sh = W.LayerShape(256, 128, 16, 8, 4, 0, 2)
+    inp = W.make_custom_inputs(sh, [6], 6, seed=10)
+    inp.slabs[0].topk_ids[:6] = [[0, 1], [8, 2], [15, -1], [-1, -1], [9, 11], [3, 4]]
+    res, ref, _ = _full_check(inp)
+    out = res["outs"][0]
+    assert np.all(out[0] == 0) and np.all(out[2] == 0) and np.all(out[3] == 0) and np.all(out[5] == 0)
+
+
+def test_bad_ids_duplicates_and_counts_set_status():
+    sh = W.LayerShape(256, 128, 8, 0, 8, 1, 3)
+    inp = W.make_custom_inputs(sh, [5, 3], 5, seed=11)
+    inp.slabs[0].topk_ids[1] = [2, 2, 9]      # repeat and out of range
+    inp.slabs[1].topk_ids[0] = [-7, 1, 3]     # negative, not -1
+    res, ref, _ = _full_check(inp)
+    assert res["status_word"] & 0x1
+    assert res["status_rc"] == 5               # AFD_ERR_BAD_ROUTING
+
+
+def test_count_above_capacity_is_clamped_and_flagged():
+    import torch
+    from attention_ffn_disaggregated_b200 import FfnLayer
+    from attention_ffn_disaggregated_b200.device import (gather_outputs, to_device_slabs,
+                                                          to_device_weights)
+    sh = W.LayerShape(256, 128, 8, 0, 8, 0, 2)
+    inp = W.make_custom_inputs(sh, [4, 4], 4, seed=12)
+    layer = FfnLayer(sh, 2, 4, *to_device_weights(inp))
+    slabs = to_device_slabs(inp)
+    layer(slabs, torch.tensor([9, 4], dtype=torch.int32, device="cuda"))
+    rc, word = layer.status()
+    assert word & 0x4 and rc == 5
+    ref = offn.ffn_layer(inp)              # counts clamp to capacity: same as [4, 4]
+    compare_outputs(gather_outputs(inp, slabs), ref["out"])
+
+
+def test_single_token_single_slab():
+    inp = W.make_custom_inputs(W.LayerShape(512, 256, 32, 0, 32, 1, 8), [1], 1, seed=13)
+    _full_check(inp)
+
+
+def test_intermediate_codes_match_oracle_mostly():
+    """Diagnostic on h: FP8 codes equal to the oracle's except rare rounding-boundary flips."""
+    inp = W.make_custom_inputs(W.LayerShape(512, 256, 8, 0, 8, 0, 2), [160, 100], 160, seed=14)
+    res = run_cuda_layer(inp)
+    ref = offn.ffn_layer(inp, keep_intermediates=True)
+    codes, scales = res["layer"].intermediate()
+    R = ref["routing"].num_rows
+    assert codes.shape == (R, 256)
+    same = codes == ref["h_codes"]
+    assert same.mean() > 0.995, same.mean()
+    np.testing.assert_allclose(scales, ref["h_scales"], rtol=1e-4)
+
+
+def test_timeout_injection_reports_status_and_recovers():
+    """A stage that is never filled makes the bounded wait expire: TIMEOUT, no hang, and
+    the next call on the same plan is correct again."""
+    inp = W.make_custom_inputs(W.LayerShape(256, 128, 8, 0, 8, 1, 2), [64], 64, seed=15)
+    res = run_cuda_layer(inp)
+    layer = res["layer"]
+    layer.set_wait_limit(50_000_000)
+    layer.inject_stall(True)
+    stalled = run_cuda_layer(inp, layer=layer)
+    assert stalled["status_word"] & 0x2 and stalled["status_rc"] == 6
+    layer.set_wait_limit(1_000_000_000)
+    again = run_cuda_layer(inp, layer=layer)
+    assert again["status_rc"] == 0
+    compare_outputs(again["outs"][0], offn.ffn_layer(inp)["out"])
+
+
+# ------------------------------------------------------------------ full-size workloads
+
+def _sampled_check(name, n_sample=40):
+    wl = W.CONFIGS[name]
+    inp = W.make_inputs(wl)
+    res = run_cuda_layer(inp)
+    assert res["status_rc"] == 0
+    ort = offn.route_inputs(inp)
+    compare_routing(res["routing"], ort)
+    rng = np.random.default_rng(0)
+    T = ort.num_tokens
+    toks = np.unique(np.concatenate([[0, T - 1], rng.choice(T, size=min(n_sample, T), replace=False)]))
+    ref = offn.ffn_layer(inp, tokens=toks, routing=ort)
+    return compare_outputs(res["outs"][0], ref["out"], tokens=toks)
+
+
+@pytest.mark.parametrize("name", ["qwen3_235b_t2048", "deepseek_v3_share_t4096",
+                                  "qwen3_235b_spec_q4_t8192"])
+def test_full_size_sampled(name):
+    _sampled_check(name)

@@ -183,7 +183,8 @@ def popularity(wl: Workload) -> np.ndarray:
 def sample_routing(wl: Workload, rng: np.random.Generator, n: int):
     """n tokens -> (ids int32 [n, K], weights f32 [n, K])."""
     K = wl.shape.top_k
-    logp = np.log(popularity(wl))           # -inf for zero-popularity ids
+    with np.errstate(divide="ignore"):
+        logp = np.log(popularity(wl))       # -inf for zero-popularity ids
     g = rng.gumbel(size=(n, logp.size))
     keys = logp[None, :] + g
     ids = np.argsort(-keys, axis=1, kind="stable")[:, :K].astype(np.int32)
