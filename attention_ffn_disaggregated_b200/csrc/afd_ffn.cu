@@ -255,8 +255,12 @@ afd_status_t afd_ffn_plan(const afd_ffn_config_t* cfg, const afd_ffn_weights_t* 
                            static_cast<int>(gemm_smem_bytes(EPI_SWIGLU))) != cudaSuccess ||
       cudaFuncSetAttribute(grouped_gemm_kernel<EPI_COMBINE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(gemm_smem_bytes(EPI_COMBINE))) != cudaSuccess ||
+      // the limit is a per-function setting shared by every plan: set the largest any
+      // configuration can need, so that a later plan never lowers an earlier plan's limit
       cudaFuncSetAttribute(route_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(std::max<size_t>(P->scatter_smem, 1))) != cudaSuccess) {
+                           static_cast<int>(sizeof(int32_t) * (kRouteWarps * AFD_MAX_GROUPS +
+                                                               kRouteWarps * 32 * AFD_MAX_TOP_K))) !=
+          cudaSuccess) {
     cudaGetLastError();
     cudaFree(P->ws);
     delete P;
