@@ -497,3 +497,127 @@ afd_status_t afd_ffn_inject_stall(afd_ffn_plan_t P, int32_t enable) {
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------------------------
+// Routing without allocation: the routing kernels run with their scratch in one
+// file-scope device array instead of a plan workspace.
+// ------------------------------------------------------------------------------------
+static __device__ __align__(256) uint8_t g_noalloc_scratch[AFD_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+uint8_t* g_noalloc_ptr[kMaxDevices] = {};
+
+// Once per device, with that device current: the array's device address (the host-side
+// name of a __device__ array is only a stand-in) and the routing scatter's shared-memory
+// limit.
+afd_status_t noalloc_setup(int dev, uint8_t** out) {
+  if (dev < 0 || dev >= kMaxDevices) return AFD_ERR_UNSUPPORTED;
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+      cudaGetLastError();
+      return AFD_ERR_CUDA;
+    }
+    if (cudaFuncSetAttribute(route_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(sizeof(int32_t) * (kRouteWarps * AFD_MAX_GROUPS +
+                                                                 kRouteWarps * 32 * AFD_MAX_TOP_K))) !=
+        cudaSuccess) {
+      cudaGetLastError();
+      return AFD_ERR_CUDA;
+    }
+    g_noalloc_ptr[dev] = static_cast<uint8_t*>(p);
+  }
+  *out = g_noalloc_ptr[dev];
+  return AFD_OK;
+}
+
+}  // namespace
+
+extern "C" afd_status_t afd_ffn_route_noalloc(const afd_ffn_config_t* cfg, const afd_slab_t* slabs,
+                                              const int32_t* d_counts, int32_t* d_sizes,
+                                              int32_t* d_group_count, int32_t* d_group_offset,
+                                              int32_t* d_row_token, int32_t* d_row_k,
+                                              float* d_row_weight, int32_t* d_pos, int32_t* d_status,
+                                              afd_stream_t stream_) {
+  afd_status_t st = afd_ffn_check_config(cfg);
+  if (st != AFD_OK) return st;
+  if (!slabs || !d_counts || !d_sizes || !d_group_count || !d_group_offset || !d_row_token ||
+      !d_row_k || !d_row_weight || !d_pos || !d_status)
+    return AFD_ERR_INVALID_ARGUMENT;
+  const afd_ffn_config_t& c = *cfg;
+  SlabTable tab;
+  memset(&tab, 0, sizeof(tab));
+  for (int m = 0; m < c.num_slabs; ++m) {
+    const afd_slab_t& s = slabs[m];
+    if (!s.topk_ids || !s.topk_weights || !s.y) return AFD_ERR_INVALID_ARGUMENT;
+    if (!aligned(s.y, 16) || !aligned(s.topk_ids, 4) || !aligned(s.topk_weights, 4))
+      return AFD_ERR_INVALID_ARGUMENT;
+    tab.ids[m] = s.topk_ids;
+    tab.w[m] = s.topk_weights;
+    tab.y[m] = static_cast<__nv_bfloat16*>(s.y);
+  }
+  // scratch layout (bytes), each region 256-byte aligned
+  const int G = c.num_local_experts + c.has_shared_expert;
+  const int El1 = std::max(c.num_local_experts, 1);
+  const int64_t tmax = static_cast<int64_t>(c.num_slabs) * c.slab_capacity;
+  const int64_t chunks = (tmax + kChunkTokens - 1) / kChunkTokens;
+  int64_t off = 0;
+  auto take = [&](int64_t bytes) {
+    const int64_t o = off;
+    off = (off + bytes + 255) / 256 * 256;
+    return o;
+  };
+  const int64_t o_base = take(4 * (c.num_slabs + 1));
+  const int64_t o_hist = take(4 * chunks * El1);
+  const int64_t o_coff = take(4 * chunks * El1);
+  const int64_t o_mtile = take(4 * (G + 1));
+  const int64_t o_tmt = take(4 * tmax);
+  const int64_t o_tneed = take(4 * tmax);
+  if (off > static_cast<int64_t>(AFD_NOALLOC_SCRATCH_BYTES)) return AFD_ERR_UNSUPPORTED;
+
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return AFD_ERR_UNSUPPORTED;
+  uint8_t* scratch = nullptr;
+  st = noalloc_setup(dev, &scratch);
+  if (st != AFD_OK) return st;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+
+  RouteParams rp;
+  memset(&rp, 0, sizeof(rp));
+  rp.counts = d_counts;
+  rp.M = c.num_slabs;
+  rp.cap = c.slab_capacity;
+  rp.K = c.top_k;
+  rp.H = c.hidden;
+  rp.e0 = c.expert_begin;
+  rp.El = c.num_local_experts;
+  rp.Eg = c.num_experts_global;
+  rp.S = c.has_shared_expert;
+  rp.G = G;
+  rp.num_chunks = static_cast<int>(chunks);
+  rp.slab_base = reinterpret_cast<int32_t*>(scratch + o_base);
+  rp.info = d_sizes;
+  rp.chunk_hist = reinterpret_cast<int32_t*>(scratch + o_hist);
+  rp.chunk_off = reinterpret_cast<int32_t*>(scratch + o_coff);
+  rp.group_count = d_group_count;
+  rp.group_off = d_group_offset;
+  rp.mtile_off = reinterpret_cast<int32_t*>(scratch + o_mtile);
+  rp.tok_mt = reinterpret_cast<int32_t*>(scratch + o_tmt);
+  rp.tok_need = reinterpret_cast<int32_t*>(scratch + o_tneed);
+  rp.pos = d_pos;
+  rp.row_token = d_row_token;
+  rp.row_k = d_row_k;
+  rp.row_w = d_row_weight;
+  rp.status = d_status;
+  // every scratch region is fully written before it is read; only the status starts at 0
+  if (cudaMemsetAsync(d_status, 0, sizeof(int32_t), stream) != cudaSuccess) return AFD_ERR_CUDA;
+  const size_t scatter_smem = sizeof(int32_t) * (static_cast<size_t>(kRouteWarps) * El1 +
+                                                 kRouteWarps * 32 * c.top_k);
+  route_count_kernel<<<static_cast<int>(chunks), kRouteThreads, 0, stream>>>(rp, tab);
+  route_scan_kernel<<<1, 1024, 0, stream>>>(rp);
+  route_scatter_kernel<<<static_cast<int>(chunks), kRouteThreads, scatter_smem, stream>>>(rp, tab);
+  if (cudaGetLastError() != cudaSuccess) return AFD_ERR_CUDA;
+  return AFD_OK;
+}

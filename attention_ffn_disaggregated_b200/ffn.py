@@ -78,6 +78,8 @@ def lib() -> ctypes.CDLL:
         "afd_ffn_set_wait_limit": (c_int32, [P, c_int64]),
         "afd_ffn_inject_stall": (c_int32, [P, c_int32]),
         "afd_ffn_kernels_per_layer": (c_int32, []),
+        "afd_ffn_route_noalloc": (c_int32, [POINTER(Config), POINTER(SlabDesc), P, P, P, P, P, P, P, P,
+                                            P, P]),
         "afd_status_string": (c_char_p, [c_int32]),
     }
     for name, (res, args) in sig.items():
@@ -217,3 +219,40 @@ class FfnLayer:
 
 def kernels_per_layer() -> int:
     return lib().afd_ffn_kernels_per_layer()
+
+
+def route_noalloc(shape, slabs: Sequence, counts, stream=None) -> dict:
+    """Routing through afd_ffn_route_noalloc: the library allocates nothing; the output
+    buffers below are allocated here, by the caller, with torch.
+
+    For callers that cannot call cudaMalloc at step time (a serving engine whose memory
+    pool already holds nearly all of HBM, a loop that must not stall on allocation).
+    Returns CUDA tensors: sizes [4] (T, R, m-tiles, 0), counts [G], offsets [G+1],
+    row_token / row_k / row_weight [max_rows], pos [M*cap*K], status [1].
+    """
+    import torch
+    M = len(slabs)
+    cap = slabs[0].topk_ids.shape[0]
+    cfg = make_config(shape, M, cap)
+    G = shape.num_local_experts + shape.has_shared_expert
+    max_rows = M * cap * (min(shape.top_k, shape.num_local_experts) + shape.has_shared_expert)
+    dev = slabs[0].topk_ids.device
+    i32 = dict(dtype=torch.int32, device=dev)
+    out = {
+        "sizes": torch.zeros(4, **i32), "counts": torch.zeros(G, **i32),
+        "offsets": torch.zeros(G + 1, **i32), "row_token": torch.zeros(max(max_rows, 1), **i32),
+        "row_k": torch.zeros(max(max_rows, 1), **i32),
+        "row_weight": torch.zeros(max(max_rows, 1), dtype=torch.float32, device=dev),
+        "pos": torch.zeros(max(M * cap * shape.top_k, 1), **i32), "status": torch.zeros(1, **i32),
+    }
+    descs = (SlabDesc * M)()
+    for i, s in enumerate(slabs):
+        descs[i] = SlabDesc(_ptr(s.x), _ptr(s.x_scale), _ptr(s.topk_ids), _ptr(s.topk_weights), _ptr(s.y))
+    P = lambda k: c_void_p(out[k].data_ptr())
+    rc = lib().afd_ffn_route_noalloc(ctypes.byref(cfg), descs, c_void_p(_ptr(counts)), P("sizes"),
+                                     P("counts"), P("offsets"), P("row_token"), P("row_k"),
+                                     P("row_weight"), P("pos"), P("status"),
+                                     c_void_p(_stream_handle(stream)))
+    if rc != AFD_OK:
+        raise AfdError(rc, "afd_ffn_route_noalloc")
+    return out

@@ -211,6 +211,42 @@ AFD_API afd_status_t afd_ffn_set_wait_limit(afd_ffn_plan_t plan, int64_t limit_n
  */
 AFD_API afd_status_t afd_ffn_inject_stall(afd_ffn_plan_t plan, int32_t enable);
 
+/*
+ * Routing without any allocation, for callers that cannot call cudaMalloc.
+ *
+ * The pages have no counterpart for this entry point; it exists for integrations where
+ * allocating at call time is not possible: a serving engine that has already reserved
+ * nearly all of HBM for its KV-cache pool, a step loop that must not stall on a
+ * synchronous allocation, or code running inside another library's callback where
+ * allocation is forbidden. It runs the routing stage of afd_ffn_layer (slab intake,
+ * histogram, scan, stable permutation) and writes the same routing arrays to caller
+ * buffers. Its scratch lives in one file-scope device array of AFD_NOALLOC_SCRATCH_BYTES
+ * bytes that every GPU which loads the library holds until the process exits.
+ *
+ * cfg, slabs (host array [num_slabs]) and d_counts: as for afd_ffn_plan/afd_ffn_layer
+ * (only topk_ids, topk_weights and y of each slab are used; y rows of tokens that receive
+ * no contribution are set to zero, as afd_ffn_layer does). Outputs, all caller-owned
+ * device memory: d_sizes int32[4] = {T, R, m-tiles, 0}; d_group_count int32[G];
+ * d_group_offset int32[G+1]; d_row_token, d_row_k int32[max_rows] and d_row_weight
+ * fp32[max_rows] (max_rows = M*cap*(min(K,E_l)+S)); d_pos int32[M*cap*K];
+ * d_status int32[1] (cleared, then OR-ed with AFD_STATUS_* bits).
+ *
+ * Returns AFD_ERR_INVALID_ARGUMENT for bad arguments, AFD_ERR_UNSUPPORTED when the
+ * configuration needs more scratch than AFD_NOALLOC_SCRATCH_BYTES, AFD_ERR_CUDA if a
+ * set-up call or launch fails. The first call on a device looks up the array's device
+ * address (cudaGetSymbolAddress) with that device current; make that first call before
+ * any stream capture. Every call shares the array and it keeps the last call's contents,
+ * so calls whose work overlaps on the GPU (different streams, or several host threads)
+ * race: order them. No cudaMalloc, cudaFree or allocating library routine is called.
+ */
+#define AFD_NOALLOC_SCRATCH_BYTES (2u << 20)
+AFD_API afd_status_t afd_ffn_route_noalloc(const afd_ffn_config_t* cfg, const afd_slab_t* slabs,
+                                           const int32_t* d_counts, int32_t* d_sizes,
+                                           int32_t* d_group_count, int32_t* d_group_offset,
+                                           int32_t* d_row_token, int32_t* d_row_k,
+                                           float* d_row_weight, int32_t* d_pos, int32_t* d_status,
+                                           afd_stream_t stream);
+
 /* Number of this library's kernels one afd_ffn_layer call launches. */
 AFD_API int32_t afd_ffn_kernels_per_layer(void);
 
