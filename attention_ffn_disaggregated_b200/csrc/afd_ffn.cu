@@ -1,11 +1,12 @@
 // Host side of the C ABI declared in include/afd_ffn.h: argument validation, workspace
 // layout, TMA descriptor encoding and the launch sequence of one layer call
-// (route count -> route scan -> route scatter -> row gather -> W13 GEMM -> W2 GEMM).
+// (route count -> route scan -> route scatter -> row gather -> W13 GEMM -> W2 GEMM ->
+// combine finalisation).
 //
 // The FFN service of an AFD deployment receives activations and routing metadata,
 // computes the FFN output and returns it (vLLM AFD plugin, "FFN service"); FastAFD runs
 // the FFN side as one persistent kernel per layer (FastAFD, "Methodology / System
-// Design", item 3). Here the work is split into six stream-ordered launches that never
+// Design", item 3). Here the work is split into seven stream-ordered launches that never
 // synchronise with the host.
 #include <cuda_runtime.h>
 #include <cuda.h>
@@ -54,7 +55,7 @@ struct afd_ffn_plan_s {
   void* ws = nullptr;
   size_t ws_bytes = 0;
   int32_t *slab_base, *info, *chunk_hist, *chunk_off, *group_count, *group_off, *mtile_off;
-  int32_t *tok_mt, *tok_need, *pos, *row_token, *row_k, *cnt;
+  int32_t *tok_mt, *tok_need, *pos, *row_token, *row_k;
   float *row_w, *sa_t, *sh_t, *acc;
   uint8_t *a_perm, *hq;
   int* status;
@@ -205,7 +206,6 @@ afd_status_t afd_ffn_plan(const afd_ffn_config_t* cfg, const afd_ffn_weights_t* 
   const size_t o_hq = take(static_cast<size_t>(P->rpad) * I, 1024);
   const size_t o_sh_t = take(sizeof(float) * static_cast<size_t>(I / 128) * P->rpad, 256);
   const size_t o_acc = take(sizeof(float) * static_cast<size_t>(P->Tmax) * H, 256);
-  const size_t o_cnt = take(sizeof(int32_t) * static_cast<size_t>(P->Tmax) * (H / 256), 256);
   P->ws_bytes = take(0, 256);
 
   if (cudaMalloc(&P->ws, P->ws_bytes) != cudaSuccess) {
@@ -238,7 +238,6 @@ afd_status_t afd_ffn_plan(const afd_ffn_config_t* cfg, const afd_ffn_weights_t* 
   P->hq = b + o_hq;
   P->sh_t = reinterpret_cast<float*>(b + o_sh_t);
   P->acc = reinterpret_cast<float*>(b + o_acc);
-  P->cnt = reinterpret_cast<int32_t*>(b + o_cnt);
 
   const int E = P->G;
   st = encode_2d(enc, &P->tm_a13, P->a_perm, H, P->rpad);
@@ -350,10 +349,7 @@ static void fill_gemm_params(afd_ffn_plan_t P, int epi, GemmParams& gp) {
     gp.ws_rows = c.hidden / 128;
     gp.row_token = P->row_token;
     gp.row_w = P->row_w;
-    gp.tok_mt = P->tok_mt;
-    gp.tok_need = P->tok_need;
     gp.acc = P->acc;
-    gp.cnt = P->cnt;
   }
 }
 
@@ -402,6 +398,8 @@ afd_status_t afd_ffn_layer(afd_ffn_plan_t P, const afd_slab_t* slabs, const int3
   grouped_gemm_kernel<EPI_COMBINE><<<P->num_sms, kGemmThreads, gemm_smem_bytes(EPI_COMBINE), stream>>>(
       g2, P->tm_a2, P->tm_w2, ytab);
   if (tm) cudaEventRecord(P->ev[6], stream);
+  combine_finalize_kernel<<<P->num_sms * 4, 256, 0, stream>>>(P->info, P->tok_mt, P->acc, c.hidden, ytab);
+  if (tm) cudaEventRecord(P->ev[7], stream);
   P->ev_valid = tm;
   if (cudaGetLastError() != cudaSuccess) return AFD_ERR_CUDA;
   return AFD_OK;

@@ -17,9 +17,8 @@
 //   SWIGLU   (W13) columns are [gate 128 | up 128] of intermediate block nt; h = silu(g)*u
 //            is requantised to e4m3 per (row, 128 channels) and stored with its scale.
 //   COMBINE  (W2)  the row's result times its top-K weight is added (fp32 reductions in
-//            L2) into the token's accumulator; the last contribution to a (token, 256
-//            columns) piece converts it to bf16, writes it into the token's slab row and
-//            clears the accumulator and counter for the next call.
+//            L2) into the token's accumulator; combine_finalize_kernel then writes every
+//            token's sum as bf16 into its slab row and clears the accumulator.
 #pragma once
 
 #include "ptx.cuh"
@@ -71,10 +70,7 @@ struct GemmParams {
   // COMBINE epilogue inputs/outputs
   const int32_t* row_token;
   const float* row_w;
-  const int32_t* tok_mt;
-  const int32_t* tok_need;
   float* acc;                 // [Tmax][H] fp32, zero between calls
-  int32_t* cnt;               // [Tmax][H/256], zero between calls
   int* status;
   unsigned long long wait_limit_ns;
   int inject_stall;
@@ -179,8 +175,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (lane == 0) {
       tma_prefetch_desc(&tm_a);
       tma_prefetch_desc(&tm_b);
+      // A rows are re-read by every column tile of their m-tile; in the down projection the
+      // weights stream past the L2-resident combine accumulators, so they go first
       const uint64_t pol_a = policy_evict_last();
-      const uint64_t pol_b = policy_evict_last();
+      const uint64_t pol_b = EPI == EPI_COMBINE ? policy_evict_first() : policy_evict_last();
       int it = 0;
       bool ok = true;
       int skipped = -1;
@@ -264,6 +262,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const uint32_t tq = tmem_base + (static_cast<uint32_t>(32 * q) << 16);
     int kbg = 0, titer = 0;
     bool ok = true;
+    const uint64_t pol_acc = policy_evict_last();
     for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x, ++titer) {
       const TileCoord c = decode_tile(tile, p.n_tiles, S.mtile, p.G, p.group_off);
       const int grow = c.row0 + trow;
@@ -282,13 +281,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       const float* ws0 = wsb + static_cast<size_t>(rs0) * p.num_kb;
       const float* ws1 = wsb + static_cast<size_t>(rs1) * p.num_kb;
-      float acc[128];
+      // acc[j] holds columns (2j, 2j+1) of this thread's 128: [0,32) from the first
+      // 64-column group, [32,64) from the second
+      float2 acc[64];
 #pragma unroll
-      for (int i = 0; i < 128; ++i) acc[i] = 0.f;
+      for (int i = 0; i < 64; ++i) acc[i] = make_float2(0.f, 0.f);
+      // scales for K block kb+1 are fetched while block kb is processed
+      const float* sap = p.sa_t + grow;
+      float sa_n = sap[0];
+      float w0_n = __ldg(ws0), w1_n = __ldg(ws1);
       for (int kb = 0; kb < p.num_kb; ++kb, ++kbg) {
-        const float sa = p.sa_t[static_cast<size_t>(kb) * p.rpad + grow];
-        const float s0 = sa * __ldg(ws0 + kb);
-        const float s1 = sa * __ldg(ws1 + kb);
+        const float s0 = sa_n * w0_n;
+        const float s1 = sa_n * w1_n;
+        if (kb + 1 < p.num_kb) {
+          sa_n = sap[static_cast<size_t>(kb + 1) * p.rpad];
+          w0_n = __ldg(ws0 + kb + 1);
+          w1_n = __ldg(ws1 + kb + 1);
+        }
         const int b = kbg & 1;
         const uint32_t tph = (kbg >> 1) & 1;
         int got = 1;
@@ -300,15 +309,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         tc_fence_after();
         const uint32_t tb = tq + b * kBN;
+        const float2 S0 = make_float2(s0, s0), S1 = make_float2(s1, s1);
         {
           float v[32], w[32];
           tmem_ld32(tb + c0, v);
           tmem_ld32(tb + c0 + 32, w);
           tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) acc[i] = fmaf(v[i], s0, acc[i]);
+          for (int i = 0; i < 16; ++i) acc[i] = __ffma2_rn(make_float2(v[2 * i], v[2 * i + 1]), S0, acc[i]);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) acc[32 + i] = fmaf(w[i], s0, acc[32 + i]);
+          for (int i = 0; i < 16; ++i)
+            acc[16 + i] = __ffma2_rn(make_float2(w[2 * i], w[2 * i + 1]), S0, acc[16 + i]);
         }
         {
           float v[32], w[32];
@@ -319,9 +330,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(&S.tempty[b]);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) acc[64 + i] = fmaf(v[i], s1, acc[64 + i]);
+          for (int i = 0; i < 16; ++i)
+            acc[32 + i] = __ffma2_rn(make_float2(v[2 * i], v[2 * i + 1]), S1, acc[32 + i]);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) acc[96 + i] = fmaf(w[i], s1, acc[96 + i]);
+          for (int i = 0; i < 16; ++i)
+            acc[48 + i] = __ffma2_rn(make_float2(w[2 * i], w[2 * i + 1]), S1, acc[48 + i]);
         }
       }
       if (!ok) break;
@@ -330,12 +343,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         // h = silu(g) * u on this thread's 64 channels; block amax shared with the partner
         // warp that holds the other 64 channels of the same rows
         float amax = 0.f;
+        float hv[64];
 #pragma unroll
-        for (int i = 0; i < 64; ++i) {
-          const float g = acc[i];
-          const float h = (g / (1.0f + expf(-g))) * acc[64 + i];
-          acc[i] = h;
-          amax = fmaxf(amax, fabsf(h));
+        for (int i = 0; i < 32; ++i) {
+          const float2 g = acc[i], u = acc[32 + i];
+          hv[2 * i] = (g.x / (1.0f + expf(-g.x))) * u.x;
+          hv[2 * i + 1] = (g.y / (1.0f + expf(-g.y))) * u.y;
+          amax = fmaxf(amax, fmaxf(fabsf(hv[2 * i]), fabsf(hv[2 * i + 1])));
         }
         float* ax = &S.amax[titer & 1][0][0];
         ax[half * kTileM + trow] = amax;
@@ -350,7 +364,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           uint4 out[4];
           uint16_t* o16 = reinterpret_cast<uint16_t*>(out);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o16[i] = pack_e4m3x2(acc[2 * i] / sc, acc[2 * i + 1] / sc);
+          for (int i = 0; i < 32; ++i) o16[i] = pack_e4m3x2(hv[2 * i] / sc, hv[2 * i + 1] / sc);
           uint4* dst = reinterpret_cast<uint4*>(p.hq + static_cast<size_t>(grow) * p.I +
                                                 c.nt * 128 + 64 * half);
 #pragma unroll
@@ -358,8 +372,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (half == 0) p.sh_t[static_cast<size_t>(c.nt) * p.rpad + grow] = sc;
         }
       } else {
-        // weighted combine: fp32 reductions into the token accumulator, staged through
-        // shared memory so that each reduction covers 128 contiguous bytes of one row
+        // weighted combine: fp32 reductions into the token accumulator (kept in L2 with
+        // an evict-last hint), staged through shared memory so that each reduction covers
+        // 128 contiguous bytes of one row; combine_finalize_kernel turns the sums into bf16
         int g = -1;
         float wgt = 0.f;
         if (valid) {
@@ -372,9 +387,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int ch = 0; ch < 8; ++ch) {
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            float4 v = make_float4(acc[16 * ch + 4 * j] * wgt, acc[16 * ch + 4 * j + 1] * wgt,
-                                   acc[16 * ch + 4 * j + 2] * wgt, acc[16 * ch + 4 * j + 3] * wgt);
-            *reinterpret_cast<float4*>(sw + lane * kStgStride + 4 * j) = v;
+            const float2 a = acc[8 * ch + 2 * j], bb = acc[8 * ch + 2 * j + 1];
+            *reinterpret_cast<float4*>(sw + lane * kStgStride + 4 * j) =
+                make_float4(a.x * wgt, a.y * wgt, bb.x * wgt, bb.y * wgt);
           }
           __syncwarp();
 #pragma unroll
@@ -384,39 +399,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const int gg = __shfl_sync(0xffffffffu, g, rr);
             const float4 v = *reinterpret_cast<const float4*>(sw + rr * kStgStride + cc);
             if (gg >= 0)
-              red_add_v4(p.acc + static_cast<size_t>(gg) * p.H + col0 + 16 * ch + cc, v.x, v.y,
-                         v.z, v.w);
+              red_add_v4_hint(p.acc + static_cast<size_t>(gg) * p.H + col0 + 16 * ch + cc, v.x,
+                              v.y, v.z, v.w, pol_acc);
           }
           __syncwarp();
-        }
-        __threadfence();
-        __syncwarp();
-        bool last = false;
-        if (g >= 0) {
-          const int old = atomicAdd(&p.cnt[static_cast<size_t>(g) * p.n_tiles + c.nt], 1);
-          last = (old == 2 * p.tok_need[g] - 1);
-        }
-        unsigned lm = __ballot_sync(0xffffffffu, last);
-        while (lm) {
-          const int src = __ffs(lm) - 1;
-          lm &= lm - 1;
-          const int gg = __shfl_sync(0xffffffffu, g, src);
-          __threadfence();
-          float* rowp = p.acc + static_cast<size_t>(gg) * p.H + c.nt * kBN + lane * 8;
-          const float4 a = ld_cg_f4(rowp);
-          const float4 bq = ld_cg_f4(rowp + 4);
-          const int mt = p.tok_mt[gg];
-          const int m = mt >> 24, t = mt & 0xFFFFFF;
-          uint4 o;
-          o.x = pack_bf16x2(a.x, a.y);
-          o.y = pack_bf16x2(a.z, a.w);
-          o.z = pack_bf16x2(bq.x, bq.y);
-          o.w = pack_bf16x2(bq.z, bq.w);
-          *reinterpret_cast<uint4*>(ytab.y[m] + static_cast<size_t>(t) * p.H + c.nt * kBN +
-                                    lane * 8) = o;
-          __stcg(reinterpret_cast<float4*>(rowp), make_float4(0.f, 0.f, 0.f, 0.f));
-          __stcg(reinterpret_cast<float4*>(rowp + 4), make_float4(0.f, 0.f, 0.f, 0.f));
-          if (lane == 0) p.cnt[static_cast<size_t>(gg) * p.n_tiles + c.nt] = 0;
         }
       }
     }
@@ -428,6 +414,35 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+// Combine, last step: every token's fp32 sum -> bf16 into its slab row; the accumulator
+// is cleared for the next call. One warp per token row, 16-byte stores.
+__global__ void __launch_bounds__(256) combine_finalize_kernel(const int32_t* __restrict__ info,
+                                                               const int32_t* __restrict__ tok_mt,
+                                                               float* __restrict__ acc, int H,
+                                                               const __grid_constant__ YTable ytab) {
+  const int T = info[0];
+  const int lane = threadIdx.x & 31;
+  const int nwarps = (gridDim.x * blockDim.x) >> 5;
+  for (int g = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; g < T; g += nwarps) {
+    const int mt = tok_mt[g];
+    const int m = mt >> 24, t = mt & 0xFFFFFF;
+    float* row = acc + static_cast<size_t>(g) * H;
+    __nv_bfloat16* y = ytab.y[m] + static_cast<size_t>(t) * H;
+    for (int c = lane * 8; c < H; c += 256) {
+      const float4 a = __ldcg(reinterpret_cast<const float4*>(row + c));
+      const float4 b = __ldcg(reinterpret_cast<const float4*>(row + c + 4));
+      uint4 o;
+      o.x = pack_bf16x2(a.x, a.y);
+      o.y = pack_bf16x2(a.z, a.w);
+      o.z = pack_bf16x2(b.x, b.y);
+      o.w = pack_bf16x2(b.z, b.w);
+      *reinterpret_cast<uint4*>(y + c) = o;
+      __stcg(reinterpret_cast<float4*>(row + c), make_float4(0.f, 0.f, 0.f, 0.f));
+      __stcg(reinterpret_cast<float4*>(row + c + 4), make_float4(0.f, 0.f, 0.f, 0.f));
+    }
   }
 }
 

@@ -234,6 +234,14 @@ __device__ __forceinline__ void red_add_v4(float* gaddr, float a, float b, float
                : "memory");
 }
 
+// fp32 vector reduction into global memory with an L2 cache-eviction hint
+__device__ __forceinline__ void red_add_v4_hint(float* gaddr, float a, float b, float c, float d,
+                                                uint64_t policy) {
+  asm volatile("red.global.add.L2::cache_hint.v4.f32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(gaddr),
+               "f"(a), "f"(b), "f"(c), "f"(d), "l"(policy)
+               : "memory");
+}
+
 __device__ __forceinline__ float4 ld_cg_f4(const float* p) {
   return __ldcg(reinterpret_cast<const float4*>(p));
 }

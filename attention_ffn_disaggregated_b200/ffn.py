@@ -22,7 +22,7 @@ STATUS_NAMES = {0: "AFD_OK", 1: "AFD_ERR_INVALID_ARGUMENT", 2: "AFD_ERR_UNSUPPOR
                 6: "AFD_ERR_TIMEOUT"}
 STATUS_BAD_ROUTING, STATUS_TIMEOUT, STATUS_BAD_COUNT = 0x1, 0x2, 0x4
 KERNEL_NAMES = ["route_count", "route_scan", "route_scatter", "gather_rows", "gemm13_swiglu",
-                "gemm2_combine"]
+                "gemm2_combine", "combine_finalize"]
 
 
 class Config(ctypes.Structure):

@@ -261,7 +261,7 @@ def main():
     torch.cuda.synchronize()
 
     kt = {k: [] for k in ("route_count", "route_scan", "route_scatter", "gather_rows",
-                          "gemm13_swiglu", "gemm2_combine")}
+                          "gemm13_swiglu", "gemm2_combine", "combine_finalize")}
     step_ms = []
     with ClockSampler(local) as clk:
         for _ in range(args.steps):

@@ -85,7 +85,8 @@ typedef enum {
 #define AFD_KERNEL_GATHER 3
 #define AFD_KERNEL_GEMM13 4
 #define AFD_KERNEL_GEMM2 5
-#define AFD_NUM_KERNELS 6
+#define AFD_KERNEL_FINALIZE 6
+#define AFD_NUM_KERNELS 7
 
 struct CUstream_st;
 typedef struct CUstream_st* afd_stream_t; /* same type as cudaStream_t; NULL = legacy stream */
