@@ -343,12 +343,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         // h = silu(g) * u on this thread's 64 channels; block amax shared with the partner
         // warp that holds the other 64 channels of the same rows
         float amax = 0.f;
+        // silu(g) = g / (1 + exp(-g)) with branch-free fast exp and division (g is
+        // clamped at -80, where silu is 0 to fp32 precision, so exp(-g) stays finite)
         float hv[64];
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           const float2 g = acc[i], u = acc[32 + i];
-          hv[2 * i] = (g.x / (1.0f + expf(-g.x))) * u.x;
-          hv[2 * i + 1] = (g.y / (1.0f + expf(-g.y))) * u.y;
+          const float gx = fmaxf(g.x, -80.0f), gy = fmaxf(g.y, -80.0f);
+          hv[2 * i] = __fdividef(gx, 1.0f + __expf(-gx)) * u.x;
+          hv[2 * i + 1] = __fdividef(gy, 1.0f + __expf(-gy)) * u.y;
           amax = fmaxf(amax, fmaxf(fabsf(hv[2 * i]), fabsf(hv[2 * i + 1])));
         }
         float* ax = &S.amax[titer & 1][0][0];
@@ -359,12 +362,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           break;
         }
         amax = fmaxf(amax, ax[(half ^ 1) * kTileM + trow]);
+        // block scale amax/448; codes = e4m3(h * (1/scale)), decided in fp32 with one
+        // correctly rounded reciprocal per row block
         const float sc = amax > 0.f ? amax / 448.0f : 1.0f;
+        const float rsc = __frcp_rn(sc);
         if (valid) {
           uint4 out[4];
           uint16_t* o16 = reinterpret_cast<uint16_t*>(out);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o16[i] = pack_e4m3x2(hv[2 * i] / sc, hv[2 * i + 1] / sc);
+          for (int i = 0; i < 32; ++i) o16[i] = pack_e4m3x2(hv[2 * i] * rsc, hv[2 * i + 1] * rsc);
           uint4* dst = reinterpret_cast<uint4*>(p.hq + static_cast<size_t>(grow) * p.I +
                                                 c.nt * 128 + 64 * half);
 #pragma unroll

@@ -309,9 +309,20 @@ __global__ void __launch_bounds__(kRouteThreads) gather_rows_kernel(
     const int g = p.row_token[r];
     const int mt = p.tok_mt[g];
     const int m = mt >> 24, t = mt & 0xFFFFFF;
-    const uint4* src = reinterpret_cast<const uint4*>(slabs.x[m] + static_cast<size_t>(t) * p.H);
-    uint4* dst = reinterpret_cast<uint4*>(p.a_perm + static_cast<size_t>(r) * p.H);
-    for (int i = lane; i < p.H / 16; i += 32) dst[i] = __ldg(src + i);
+    const uint4* __restrict__ src =
+        reinterpret_cast<const uint4*>(slabs.x[m] + static_cast<size_t>(t) * p.H);
+    uint4* __restrict__ dst = reinterpret_cast<uint4*>(p.a_perm + static_cast<size_t>(r) * p.H);
+    const int n16 = p.H / 16;             // H is a multiple of 256: n16 a multiple of 16
+    int i = lane;
+    for (; i + 96 < n16; i += 128) {      // four 16-byte loads in flight per lane
+      const uint4 a = __ldg(src + i), b = __ldg(src + i + 32), c = __ldg(src + i + 64),
+                  d = __ldg(src + i + 96);
+      dst[i] = a;
+      dst[i + 32] = b;
+      dst[i + 64] = c;
+      dst[i + 96] = d;
+    }
+    for (; i < n16; i += 32) dst[i] = __ldg(src + i);
     const float* ssrc = slabs.xs[m] + static_cast<size_t>(t) * KB;
     for (int kb = lane; kb < KB; kb += 32) p.sa_t[static_cast<size_t>(kb) * p.rpad + r] = ssrc[kb];
   }
