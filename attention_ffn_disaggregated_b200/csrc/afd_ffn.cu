@@ -54,7 +54,9 @@ struct afd_ffn_plan_s {
   int G = 0, Tmax = 0, Rmax = 0, rpad = 0, num_chunks = 0;
   void* ws = nullptr;
   size_t ws_bytes = 0;
-  int32_t *slab_base, *info, *chunk_hist, *chunk_off, *group_count, *group_off, *mtile_off;
+  int32_t *slab_base, *info, *chunk_hist, *chunk_off, *group_count, *group_off, *mtile_off,
+      *mtile2_off;
+  int tiling = 0;  // 0 = chosen per call on the device; 1 / 2 forced
   int32_t *tok_mt, *tok_need, *pos, *row_token, *row_k;
   float *row_w, *sa_t, *sh_t, *acc;
   uint8_t *a_perm, *hq;
@@ -82,7 +84,8 @@ const char* afd_status_string(afd_status_t s) {
   return "unknown";
 }
 
-int32_t afd_ffn_kernels_per_layer(void) { return AFD_NUM_KERNELS; }
+// route count, scan, scatter, gather, W13 (two tilings), W2 (two tilings), finalize
+int32_t afd_ffn_kernels_per_layer(void) { return 9; }
 
 afd_status_t afd_ffn_check_config(const afd_ffn_config_t* c) {
   if (!c) return AFD_ERR_INVALID_ARGUMENT;
@@ -124,10 +127,10 @@ static afd_status_t encode_2d(EncodeTiledFn enc, CUtensorMap* m, void* base, uin
 }
 
 static afd_status_t encode_3d(EncodeTiledFn enc, CUtensorMap* m, const void* base, uint64_t inner,
-                              uint64_t rows, uint64_t experts) {
+                              uint64_t rows, uint64_t experts, uint32_t box_rows) {
   cuuint64_t dims[3] = {inner, rows, experts};
   cuuint64_t strides[2] = {inner, inner * rows};
-  cuuint32_t box[3] = {128, 128, 1};
+  cuuint32_t box[3] = {128, box_rows, 1};
   cuuint32_t es[3] = {1, 1, 1};
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides,
                    box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -156,12 +159,16 @@ afd_status_t afd_ffn_plan(const afd_ffn_config_t* cfg, const afd_ffn_weights_t* 
   if (!enc) return AFD_ERR_CUDA;
   // The GEMM kernels split the block's registers between warpgroups with setmaxnreg; that
   // is only safe when the block is launched with exactly the budget the split assumes.
-  for (int epi = 0; epi < 2; ++epi) {
-    cudaFuncAttributes fa;
-    cudaError_t e = epi == 0 ? cudaFuncGetAttributes(&fa, grouped_gemm_kernel<EPI_SWIGLU>)
-                             : cudaFuncGetAttributes(&fa, grouped_gemm_kernel<EPI_COMBINE>);
-    if (e != cudaSuccess) return AFD_ERR_CUDA;
-    if (fa.numRegs != kLaunchRegs || fa.maxThreadsPerBlock < kGemmThreads) return AFD_ERR_UNSUPPORTED;
+  {
+    const void* fns[4] = {reinterpret_cast<const void*>(grouped_gemm_kernel<EPI_SWIGLU, 1>),
+                          reinterpret_cast<const void*>(grouped_gemm_kernel<EPI_SWIGLU, 2>),
+                          reinterpret_cast<const void*>(grouped_gemm_kernel<EPI_COMBINE, 1>),
+                          reinterpret_cast<const void*>(grouped_gemm_kernel<EPI_COMBINE, 2>)};
+    for (const void* fn : fns) {
+      cudaFuncAttributes fa;
+      if (cudaFuncGetAttributes(&fa, fn) != cudaSuccess) return AFD_ERR_CUDA;
+      if (fa.numRegs != kLaunchRegs || fa.maxThreadsPerBlock < kGemmThreads) return AFD_ERR_UNSUPPORTED;
+    }
   }
 
   afd_ffn_plan_s* P = new (std::nothrow) afd_ffn_plan_s();
@@ -175,7 +182,8 @@ afd_status_t afd_ffn_plan(const afd_ffn_config_t* cfg, const afd_ffn_weights_t* 
   P->G = El + S;
   P->Tmax = cfg->num_slabs * cfg->slab_capacity;
   P->Rmax = P->Tmax * (std::min(K, El) + S);
-  P->rpad = ((P->Rmax + 128 + 127) / 128) * 128;
+  // a CTA-pair tile may start up to 255 rows before the end of the routed rows
+  P->rpad = ((P->Rmax + 256 + 127) / 128) * 128;
   P->num_chunks = (P->Tmax + kChunkTokens - 1) / kChunkTokens;
   const int El1 = std::max(El, 1);
 
@@ -195,6 +203,7 @@ afd_status_t afd_ffn_plan(const afd_ffn_config_t* cfg, const afd_ffn_weights_t* 
   const size_t o_group_count = take(sizeof(int32_t) * (P->G + 1), 16);
   const size_t o_group_off = take(sizeof(int32_t) * (P->G + 1), 16);
   const size_t o_mtile_off = take(sizeof(int32_t) * (P->G + 1), 16);
+  const size_t o_mtile2_off = take(sizeof(int32_t) * (P->G + 1), 16);
   const size_t o_tok_mt = take(sizeof(int32_t) * P->Tmax, 16);
   const size_t o_tok_need = take(sizeof(int32_t) * P->Tmax, 16);
   const size_t o_pos = take(sizeof(int32_t) * static_cast<size_t>(P->Tmax) * K, 16);
@@ -227,6 +236,7 @@ afd_status_t afd_ffn_plan(const afd_ffn_config_t* cfg, const afd_ffn_weights_t* 
   P->group_count = reinterpret_cast<int32_t*>(b + o_group_count);
   P->group_off = reinterpret_cast<int32_t*>(b + o_group_off);
   P->mtile_off = reinterpret_cast<int32_t*>(b + o_mtile_off);
+  P->mtile2_off = reinterpret_cast<int32_t*>(b + o_mtile2_off);
   P->tok_mt = reinterpret_cast<int32_t*>(b + o_tok_mt);
   P->tok_need = reinterpret_cast<int32_t*>(b + o_tok_need);
   P->pos = reinterpret_cast<int32_t*>(b + o_pos);
@@ -241,18 +251,23 @@ afd_status_t afd_ffn_plan(const afd_ffn_config_t* cfg, const afd_ffn_weights_t* 
 
   const int E = P->G;
   st = encode_2d(enc, &P->tm_a13, P->a_perm, H, P->rpad);
-  if (st == AFD_OK) st = encode_3d(enc, &P->tm_w13, weights->w13, H, 2 * static_cast<uint64_t>(I), E);
+  if (st == AFD_OK) st = encode_3d(enc, &P->tm_w13, weights->w13, H, 2 * static_cast<uint64_t>(I), E, 128);
   if (st == AFD_OK) st = encode_2d(enc, &P->tm_a2, P->hq, I, P->rpad);
-  if (st == AFD_OK) st = encode_3d(enc, &P->tm_w2, weights->w2, I, H, E);
+  if (st == AFD_OK) st = encode_3d(enc, &P->tm_w2, weights->w2, I, H, E, 128);
+
   if (st != AFD_OK) {
     cudaFree(P->ws);
     delete P;
     return st;
   }
   P->scatter_smem = sizeof(int32_t) * (static_cast<size_t>(kRouteWarps) * El1 + kRouteWarps * 32 * K);
-  if (cudaFuncSetAttribute(grouped_gemm_kernel<EPI_SWIGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (cudaFuncSetAttribute(grouped_gemm_kernel<EPI_SWIGLU, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(gemm_smem_bytes(EPI_SWIGLU))) != cudaSuccess ||
-      cudaFuncSetAttribute(grouped_gemm_kernel<EPI_COMBINE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      cudaFuncSetAttribute(grouped_gemm_kernel<EPI_SWIGLU, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(gemm_smem_bytes(EPI_SWIGLU))) != cudaSuccess ||
+      cudaFuncSetAttribute(grouped_gemm_kernel<EPI_COMBINE, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(gemm_smem_bytes(EPI_COMBINE))) != cudaSuccess ||
+      cudaFuncSetAttribute(grouped_gemm_kernel<EPI_COMBINE, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(gemm_smem_bytes(EPI_COMBINE))) != cudaSuccess ||
       // the limit is a per-function setting shared by every plan: set the largest any
       // configuration can need, so that a later plan never lowers an earlier plan's limit
@@ -289,6 +304,25 @@ afd_status_t afd_ffn_get_info(afd_ffn_plan_t P, afd_ffn_plan_info_t* info) {
   return AFD_OK;
 }
 
+// Launch a CTA-pair kernel: clusters of two consecutive CTAs.
+static cudaError_t launch_pair(void (*kernel)(GemmParams, CUtensorMap, CUtensorMap, YTable), int grid,
+                               size_t smem, cudaStream_t stream, const GemmParams& gp,
+                               const CUtensorMap& ta, const CUtensorMap& tb, const YTable& ytab) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(kGemmThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, gp, ta, tb, ytab);
+}
+
 static void fill_route_params(afd_ffn_plan_t P, const int32_t* d_counts, RouteParams& rp) {
   const afd_ffn_config_t& c = P->cfg;
   rp.counts = d_counts;
@@ -310,6 +344,8 @@ static void fill_route_params(afd_ffn_plan_t P, const int32_t* d_counts, RoutePa
   rp.group_count = P->group_count;
   rp.group_off = P->group_off;
   rp.mtile_off = P->mtile_off;
+  rp.mtile2_off = P->mtile2_off;
+  rp.tiling = P->tiling;
   rp.tok_mt = P->tok_mt;
   rp.tok_need = P->tok_need;
   rp.pos = P->pos;
@@ -324,8 +360,10 @@ static void fill_route_params(afd_ffn_plan_t P, const int32_t* d_counts, RoutePa
 static void fill_gemm_params(afd_ffn_plan_t P, int epi, GemmParams& gp) {
   const afd_ffn_config_t& c = P->cfg;
   memset(&gp, 0, sizeof(gp));
+  gp.info = P->info;
   gp.group_off = P->group_off;
   gp.mtile_off = P->mtile_off;
+  gp.mtile2_off = P->mtile2_off;
   gp.G = P->G;
   gp.rpad = P->rpad;
   gp.I = c.intermediate;
@@ -392,11 +430,19 @@ afd_status_t afd_ffn_layer(afd_ffn_plan_t P, const afd_slab_t* slabs, const int3
   if (tm) cudaEventRecord(P->ev[3], stream);
   gather_rows_kernel<<<P->num_sms * 4, kRouteThreads, 0, stream>>>(rp, tab);
   if (tm) cudaEventRecord(P->ev[4], stream);
-  grouped_gemm_kernel<EPI_SWIGLU><<<P->num_sms, kGemmThreads, gemm_smem_bytes(EPI_SWIGLU), stream>>>(
+  // both tilings are launched; the one the routing scan did not choose exits at entry
+  const int grid1 = P->num_sms, grid2 = P->num_sms & ~1;
+  grouped_gemm_kernel<EPI_SWIGLU, 1><<<grid1, kGemmThreads, gemm_smem_bytes(EPI_SWIGLU), stream>>>(
       g13, P->tm_a13, P->tm_w13, ytab);
+  if (launch_pair(grouped_gemm_kernel<EPI_SWIGLU, 2>, grid2, gemm_smem_bytes(EPI_SWIGLU), stream, g13,
+                  P->tm_a13, P->tm_w13, ytab) != cudaSuccess)
+    return AFD_ERR_CUDA;
   if (tm) cudaEventRecord(P->ev[5], stream);
-  grouped_gemm_kernel<EPI_COMBINE><<<P->num_sms, kGemmThreads, gemm_smem_bytes(EPI_COMBINE), stream>>>(
+  grouped_gemm_kernel<EPI_COMBINE, 1><<<grid1, kGemmThreads, gemm_smem_bytes(EPI_COMBINE), stream>>>(
       g2, P->tm_a2, P->tm_w2, ytab);
+  if (launch_pair(grouped_gemm_kernel<EPI_COMBINE, 2>, grid2, gemm_smem_bytes(EPI_COMBINE), stream, g2,
+                  P->tm_a2, P->tm_w2, ytab) != cudaSuccess)
+    return AFD_ERR_CUDA;
   if (tm) cudaEventRecord(P->ev[6], stream);
   combine_finalize_kernel<<<P->num_sms * 4, 256, 0, stream>>>(P->info, P->tok_mt, P->acc, c.hidden, ytab);
   if (tm) cudaEventRecord(P->ev[7], stream);
@@ -485,6 +531,20 @@ afd_status_t afd_ffn_get_kernel_times(afd_ffn_plan_t P, float* ms) {
 afd_status_t afd_ffn_set_wait_limit(afd_ffn_plan_t P, int64_t limit_ns) {
   if (!P || limit_ns <= 0) return AFD_ERR_INVALID_ARGUMENT;
   P->wait_limit_ns = static_cast<unsigned long long>(limit_ns);
+  return AFD_OK;
+}
+
+afd_status_t afd_ffn_set_tiling(afd_ffn_plan_t P, int32_t tiling) {
+  if (!P || tiling < 0 || tiling > 2) return AFD_ERR_INVALID_ARGUMENT;
+  P->tiling = tiling;
+  return AFD_OK;
+}
+
+afd_status_t afd_ffn_get_tiling(afd_ffn_plan_t P, afd_stream_t stream, int32_t* tiling) {
+  if (!P || !tiling) return AFD_ERR_INVALID_ARGUMENT;
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return AFD_ERR_CUDA;
+  if (cudaMemcpy(tiling, P->info + 3, sizeof(int32_t), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return AFD_ERR_CUDA;
   return AFD_OK;
 }
 
@@ -602,6 +662,7 @@ extern "C" afd_status_t afd_ffn_route_noalloc(const afd_ffn_config_t* cfg, const
   rp.group_count = d_group_count;
   rp.group_off = d_group_offset;
   rp.mtile_off = reinterpret_cast<int32_t*>(scratch + o_mtile);
+  rp.mtile2_off = nullptr;
   rp.tok_mt = reinterpret_cast<int32_t*>(scratch + o_tmt);
   rp.tok_need = reinterpret_cast<int32_t*>(scratch + o_tneed);
   rp.pos = d_pos;

@@ -2,16 +2,26 @@
 // expert projections of the FFN-pool layer (FastAFD, "Methodology / System Design",
 // item 3: "block-FP8 grouped GEMMs, activation and push-back").
 //
-// Tile: 128 routed rows of one expert x 256 output columns, K in blocks of 128 (the
-// quantisation block). Each 128-wide K block is one tcgen05 partial product
+// Output tile per CTA: 128 routed rows of one expert x 256 output columns; K runs in
+// blocks of 128 (the quantisation block). Each K block is one tcgen05 partial product
 // (4 x kind::f8f6f4 MMAs of K=32) into one of two TMEM buffers; the epilogue warps read
 // the partial, multiply it by (row scale x weight-block scale) and accumulate in fp32
 // registers ("software promotion": the scales are arbitrary fp32, so they cannot ride on
 // the hardware's UE8M0 block-scale path).
 //
-// Warp roles (384 threads): warp 0 issues TMA loads, warp 1 owns TMEM and issues MMAs,
-// warps 2..3 idle, warps 4..11 are the epilogue (two per TMEM lane quadrant, splitting
-// the columns).
+// Two tilings (the routing scan records which one a call uses; see route_scan_kernel):
+//   PAIR = 1  one CTA per tile; per K block it loads A 128x128 and B 256x128 (48 KiB).
+//   PAIR = 2  a CTA pair (cluster of two) shares a 256-row tile of one expert: each CTA
+//             loads its own 128 A rows and half of B (32 KiB per K block), the leader
+//             issues cta_group::2 MMAs (M = 256) and each CTA's TMEM receives its rows.
+//             Less operand traffic per MMA and 6 pipeline stages instead of 4, but each
+//             K block needs a partial-ready / partial-drained handshake between the two
+//             SMs; with only one K block of TMEM slack that latency is exposed, and on
+//             the measured workloads this tiling is about 2x slower. Opt-in only.
+//
+// Warp roles (384 threads): warp 0 issues TMA loads, warp 1 owns TMEM and (leader) issues
+// MMAs, warps 2..3 idle, warps 4..11 are the epilogue (two per TMEM lane quadrant,
+// splitting the columns).
 //
 // Epilogues:
 //   SWIGLU   (W13) columns are [gate 128 | up 128] of intermediate block nt; h = silu(g)*u
@@ -26,10 +36,14 @@
 
 namespace afd {
 
-constexpr int kStages = 4;
 constexpr int kBN = 256;
 constexpr int kBK = 128;
 constexpr int kGemmThreads = 384;
+constexpr int kEpiWarps = 8;
+constexpr uint32_t kABytes = kTileM * kBK;   // 16 KiB: 128 rows of one K block
+constexpr int kStgStride = 20;               // floats per staging row (16 + 4 pad)
+constexpr uint32_t kTmemCols = 512;          // two 256-column fp32 partial buffers
+constexpr int kMaxStages = 6;
 // Register split: the block launches with kLaunchRegs per thread; warpgroup 0 (TMA, MMA,
 // two idle warps) drops to kProducerRegs and the two epilogue warpgroups rise to
 // kEpilogueRegs. 128*40 + 256*232 == 384*168, so the increase never waits for registers
@@ -39,22 +53,27 @@ constexpr int kProducerRegs = 40;
 constexpr int kEpilogueRegs = 232;
 static_assert(128 * kProducerRegs + 256 * kEpilogueRegs <= kGemmThreads * kLaunchRegs,
               "register split exceeds the launch allocation");
-constexpr int kEpiWarps = 8;
-constexpr uint32_t kABytes = kTileM * kBK;   // 16 KiB
-constexpr uint32_t kBBytes = kBN * kBK;      // 32 KiB
-constexpr uint32_t kStageBytes = kABytes + kBBytes;
-constexpr int kStgStride = 20;               // floats per staging row (16 + 4 pad)
-constexpr uint32_t kTmemCols = 512;          // two 256-column fp32 partial buffers
 
 enum EpiKind { EPI_SWIGLU = 0, EPI_COMBINE = 1 };
+
+template <int PAIR>
+struct Tiling {
+  static constexpr int kStages = PAIR == 2 ? 6 : 4;
+  static constexpr uint32_t kBBytes = (kBN / PAIR) * kBK;     // B rows held by this CTA
+  static constexpr uint32_t kStageBytes = kABytes + kBBytes;  // per CTA
+  static constexpr uint32_t kTxBytes = PAIR * kStageBytes;    // landing on the leader's barrier
+  static constexpr int kRows = PAIR * kTileM;                 // rows of one (pair) tile
+};
 
 struct YTable {
   __nv_bfloat16* y[AFD_MAX_SLABS];
 };
 
 struct GemmParams {
+  const int32_t* info;        // [3] = tiling chosen for this call (1 or 2)
   const int32_t* group_off;   // [G+1] first row of each group
-  const int32_t* mtile_off;   // [G+1] first m-tile of each group
+  const int32_t* mtile_off;   // [G+1] first 128-row m-tile of each group
+  const int32_t* mtile2_off;  // [G+1] first 256-row m-tile of each group
   int G;
   int n_tiles;                // 256-column tiles per m-tile
   int num_kb;                 // K blocks of 128
@@ -77,8 +96,8 @@ struct GemmParams {
 };
 
 struct GemmSmem {
-  uint64_t full[kStages];
-  uint64_t empty[kStages];
+  uint64_t full[kMaxStages];
+  uint64_t empty[kMaxStages];
   uint64_t tfull[2];
   uint64_t tempty[2];
   uint64_t pair[4];           // SWIGLU: amax exchange between the two warps of a quadrant
@@ -88,7 +107,9 @@ struct GemmSmem {
   int32_t mtile[AFD_MAX_GROUPS + 1];
 };
 
-constexpr size_t kGemmSmemTiles = static_cast<size_t>(kStages) * kStageBytes;
+constexpr size_t kGemmSmemTiles = static_cast<size_t>(192) * 1024;   // both tilings
+static_assert(Tiling<1>::kStages * Tiling<1>::kStageBytes == kGemmSmemTiles, "tiling size");
+static_assert(Tiling<2>::kStages * Tiling<2>::kStageBytes == kGemmSmemTiles, "tiling size");
 constexpr size_t kStgBytes = static_cast<size_t>(kEpiWarps) * 32 * kStgStride * sizeof(float);
 
 __host__ __device__ constexpr size_t gemm_smem_bytes(int epi) {
@@ -108,8 +129,11 @@ struct TileCoord {
   int e, row0, rows, nt;
 };
 
+// Tile -> (expert, first row of this CTA's 128 rows, valid rows, column tile).
+// `rows` may be <= 0 for the second CTA of a pair on an expert's last tile.
+template <int PAIR>
 __device__ __forceinline__ TileCoord decode_tile(int tile, int n_tiles, const int32_t* s_mtile,
-                                                 int G, const int32_t* group_off) {
+                                                 int G, const int32_t* group_off, int rank) {
   TileCoord c;
   const int mt = tile / n_tiles;
   c.nt = tile - mt * n_tiles;
@@ -120,17 +144,22 @@ __device__ __forceinline__ TileCoord decode_tile(int tile, int n_tiles, const in
   }
   c.e = lo;
   const int g0 = group_off[lo], g1 = group_off[lo + 1];
-  c.row0 = g0 + (mt - s_mtile[lo]) * kTileM;
+  c.row0 = g0 + (mt - s_mtile[lo]) * Tiling<PAIR>::kRows + rank * kTileM;
   c.rows = min(kTileM, g1 - c.row0);
   return c;
 }
 
-template <int EPI>
+template <int EPI, int PAIR>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ GemmParams p,
                         const __grid_constant__ CUtensorMap tm_a,
                         const __grid_constant__ CUtensorMap tm_b,
                         const __grid_constant__ YTable ytab) {
+  using TL = Tiling<PAIR>;
+  constexpr int kStages = TL::kStages;
+  // only the tiling the routing stage chose for this call runs; the other launch exits
+  if (p.info[3] != PAIR) return;
+
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -142,6 +171,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   volatile int* abort_flag = &S.abort_flag;
+  const uint32_t rank = PAIR == 2 ? cluster_ctarank() : 0;
+  const bool leader = rank == 0;
+  const int unit = PAIR == 2 ? blockIdx.x / 2 : blockIdx.x;    // pair (or CTA) index
+  const int nunits = PAIR == 2 ? gridDim.x / 2 : gridDim.x;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -150,19 +183,26 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&S.tfull[b], 1);
-      mbar_init(&S.tempty[b], kEpiWarps);
+      mbar_init(&S.tempty[b], kEpiWarps * PAIR);
     }
     for (int i = 0; i < 4; ++i) mbar_init(&S.pair[i], 64);
     S.abort_flag = 0;
     fence_mbar_init();
   }
-  for (int i = threadIdx.x; i <= p.G; i += blockDim.x) S.mtile[i] = p.mtile_off[i];
+  const int32_t* mtile_src = PAIR == 2 ? p.mtile2_off : p.mtile_off;
+  for (int i = threadIdx.x; i <= p.G; i += blockDim.x) S.mtile[i] = mtile_src[i];
   if (warp == 1) {
-    tmem_alloc(&S.tmem_base, kTmemCols);
-    tmem_relinquish();
+    if (PAIR == 2) {
+      tmem_alloc_pair(&S.tmem_base, kTmemCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(&S.tmem_base, kTmemCols);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
+  if (PAIR == 2) cluster_sync();     // both CTAs' barriers exist before any remote signal
   tc_fence_after();
   const uint32_t tmem_base = S.tmem_base;
   const int total_tiles = S.mtile[p.G] * p.n_tiles;
@@ -170,20 +210,28 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp < 4) {
     // each role's code sits inside the branch that sets its register budget
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kProducerRegs));
-    if (warp == 0) {
-    // ------------------------------------------------------------------ TMA producer
-    if (lane == 0) {
+    if (warp == 0 && lane == 0) {
+      // ---------------------------------------------------------------- TMA producer
       tma_prefetch_desc(&tm_a);
       tma_prefetch_desc(&tm_b);
-      // A rows are re-read by every column tile of their m-tile; in the down projection the
-      // weights stream past the L2-resident combine accumulators, so they go first
+      // A rows are re-read by every column tile of their m-tile; in the down projection
+      // the weights stream past the L2-resident combine accumulators, so they go first
       const uint64_t pol_a = policy_evict_last();
       const uint64_t pol_b = EPI == EPI_COMBINE ? policy_evict_first() : policy_evict_last();
       int it = 0;
       bool ok = true;
       int skipped = -1;
-      for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
-        const TileCoord c = decode_tile(tile, p.n_tiles, S.mtile, p.G, p.group_off);
+      for (int tile = unit; ok && tile < total_tiles; tile += nunits) {
+        const TileCoord c = decode_tile<PAIR>(tile, p.n_tiles, S.mtile, p.G, p.group_off, rank);
+        // B rows of this tile: [brow0, +128) and [brow1, +128); a pair splits them
+        int brow0, brow1;
+        if (EPI == EPI_SWIGLU) {
+          brow0 = c.nt * 128;               // gate block
+          brow1 = p.I + c.nt * 128;         // up block
+        } else {
+          brow0 = c.nt * kBN;
+          brow1 = c.nt * kBN + 128;
+        }
         for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
           const int s = it % kStages;
           const uint32_t ph = (it / kStages) & 1;
@@ -195,33 +243,34 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             skipped = it;       // test hook: never fill this stage
             continue;
           }
-          mbar_arrive_expect_tx(&S.full[s], kStageBytes);
-          tma_load_2d(sA + s * kABytes, &tm_a, &S.full[s], kb * kBK, c.row0, pol_a);
-          uint8_t* b = sB + s * kBBytes;
-          if (EPI == EPI_SWIGLU) {
-            tma_load_3d(b, &tm_b, &S.full[s], kb * kBK, c.nt * 128, c.e, pol_b);
-            tma_load_3d(b + kBBytes / 2, &tm_b, &S.full[s], kb * kBK, p.I + c.nt * 128, c.e, pol_b);
+          uint8_t* a = sA + s * kABytes;
+          uint8_t* b = sB + s * TL::kBBytes;
+          if (PAIR == 1) {
+            mbar_arrive_expect_tx(&S.full[s], TL::kTxBytes);
+            tma_load_2d(a, &tm_a, &S.full[s], kb * kBK, c.row0, pol_a);
+            tma_load_3d(b, &tm_b, &S.full[s], kb * kBK, brow0, c.e, pol_b);
+            tma_load_3d(b + TL::kBBytes / 2, &tm_b, &S.full[s], kb * kBK, brow1, c.e, pol_b);
           } else {
-            tma_load_3d(b, &tm_b, &S.full[s], kb * kBK, c.nt * kBN, c.e, pol_b);
-            tma_load_3d(b + kBBytes / 2, &tm_b, &S.full[s], kb * kBK, c.nt * kBN + 128, c.e, pol_b);
+            const uint32_t fb = mapa_shared(smem_u32(&S.full[s]), 0);
+            if (leader) mbar_arrive_expect_tx(&S.full[s], TL::kTxBytes);
+            tma_load_2d_pair(a, &tm_a, fb, kb * kBK, c.row0, pol_a);
+            tma_load_3d_pair(b, &tm_b, fb, kb * kBK, leader ? brow0 : brow1, c.e, pol_b);
           }
         }
       }
-      if (!ok) {
-        // wait (bounded) for the copies this thread issued that may still be landing
+      if (!ok && leader) {
+        // wait (bounded) for copies that may still be landing on this CTA's barriers
         for (int j = max(0, it - kStages); j < it; ++j) {
           if (j == skipped) continue;
           mbar_wait_drain(&S.full[j % kStages], (j / kStages) & 1, p.wait_limit_ns);
         }
       }
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_e4m3_f32(kTileM, kBN);
+    } else if (warp == 1 && lane == 0 && leader) {
+      // ---------------------------------------------------------------- MMA issuer
+      constexpr uint32_t idesc = idesc_e4m3_f32(TL::kRows, kBN);
       int it = 0, kbg = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
+      for (int tile = unit; ok && tile < total_tiles; tile += nunits) {
         for (int kb = 0; kb < p.num_kb; ++kb, ++it, ++kbg) {
           const int s = it % kStages;
           const uint32_t ph = (it / kStages) & 1;
@@ -231,26 +280,42 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
           const int b = kbg & 1;
           const uint32_t tph = (kbg >> 1) & 1;
-          if (!mbar_wait(&S.tempty[b], tph ^ 1, abort_flag, p.status, p.wait_limit_ns)) {
+          const bool got = PAIR == 2
+                               ? mbar_wait_cluster(&S.tempty[b], tph ^ 1, abort_flag, p.status,
+                                                   p.wait_limit_ns)
+                               : mbar_wait(&S.tempty[b], tph ^ 1, abort_flag, p.status,
+                                           p.wait_limit_ns);
+          if (!got) {
             ok = false;
             break;
           }
           tc_fence_after();
           const uint32_t d = tmem_base + b * kBN;
           const uint64_t a0 = sdesc_k_sw128(smem_u32(sA + s * kABytes));
-          const uint64_t b0 = sdesc_k_sw128(smem_u32(sB + s * kBBytes));
+          const uint64_t b0 = sdesc_k_sw128(smem_u32(sB + s * TL::kBBytes));
+          if (PAIR == 1) {
 #pragma unroll
-          for (int k = 0; k < kBK / 32; ++k)
-            umma_e4m3(d, a0 + 2 * k, b0 + 2 * k, idesc, k > 0 ? 1u : 0u);
-          umma_commit(&S.empty[s]);
-          umma_commit(&S.tfull[b]);
+            for (int k = 0; k < kBK / 32; ++k)
+              umma_e4m3(d, a0 + 2 * k, b0 + 2 * k, idesc, k > 0 ? 1u : 0u);
+            umma_commit(&S.empty[s]);
+            umma_commit(&S.tfull[b]);
+          } else {
+#pragma unroll
+            for (int k = 0; k < kBK / 32; ++k)
+              umma_e4m3_pair(d, a0 + 2 * k, b0 + 2 * k, idesc, k > 0 ? 1u : 0u);
+            // the same barriers in both CTAs: this CTA's and the peer's copy
+            const uint32_t e_own = smem_u32(&S.empty[s]), t_own = smem_u32(&S.tfull[b]);
+            umma_commit_pair(e_own);
+            umma_commit_pair(mapa_shared(e_own, 1));
+            umma_commit_pair(t_own);
+            umma_commit_pair(mapa_shared(t_own, 1));
+          }
         }
       }
       if (!ok && kbg > 0) {
         const int last = kbg - 1;
         mbar_wait_drain(&S.tfull[last & 1], (last >> 1) & 1, p.wait_limit_ns);
       }
-    }
     }
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kEpilogueRegs));
@@ -260,11 +325,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int q = warp & 3;                 // TMEM lane quadrant this warp may access
     const int trow = 32 * q + lane;
     const uint32_t tq = tmem_base + (static_cast<uint32_t>(32 * q) << 16);
+    // the MMA issuer waits on the leader's tempty barriers
+    const uint32_t tempty0 = PAIR == 2 ? mapa_shared(smem_u32(&S.tempty[0]), 0) : 0u;
+    const uint32_t tempty1 = PAIR == 2 ? mapa_shared(smem_u32(&S.tempty[1]), 0) : 0u;
     int kbg = 0, titer = 0;
     bool ok = true;
     const uint64_t pol_acc = policy_evict_last();
-    for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x, ++titer) {
-      const TileCoord c = decode_tile(tile, p.n_tiles, S.mtile, p.G, p.group_off);
+    for (int tile = unit; ok && tile < total_tiles; tile += nunits, ++titer) {
+      const TileCoord c = decode_tile<PAIR>(tile, p.n_tiles, S.mtile, p.G, p.group_off, rank);
       const int grow = c.row0 + trow;
       const bool valid = trow < c.rows;
       const float* wsb = p.w_scale + static_cast<size_t>(c.e) * p.ws_rows * p.num_kb;
@@ -328,7 +396,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tmem_wait_ld();
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&S.tempty[b]);
+          if (lane == 0) {
+            if (PAIR == 2) mbar_arrive_cluster(b ? tempty1 : tempty0);
+            else mbar_arrive(&S.tempty[b]);
+          }
 #pragma unroll
           for (int i = 0; i < 16; ++i)
             acc[32 + i] = __ffma2_rn(make_float2(v[2 * i], v[2 * i + 1]), S1, acc[32 + i]);
@@ -416,10 +487,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   tc_fence_before();
   __syncthreads();
+  // neither CTA of a pair leaves while the other may still signal its barriers
+  if (PAIR == 2) cluster_sync();
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_base, kTmemCols);
+    if (PAIR == 2) tmem_dealloc_pair(tmem_base, kTmemCols);
+    else tmem_dealloc(tmem_base, kTmemCols);
   }
 }
 

@@ -38,7 +38,9 @@ struct RouteParams {
   int32_t* chunk_off;     // [num_chunks][max(El,1)]
   int32_t* group_count;   // [G]
   int32_t* group_off;     // [G+1]
-  int32_t* mtile_off;     // [G+1]
+  int32_t* mtile_off;     // [G+1] 128-row m-tiles
+  int32_t* mtile2_off;    // [G+1] 256-row m-tiles (CTA-pair tiling); may be null
+  int tiling;             // 0: choose per call from the counts; 1 or 2: forced
   int32_t* tok_mt;        // [Tmax] (slab << 24) | row
   int32_t* tok_need;      // [Tmax] contributions this GPU adds to the token
   int32_t* pos;           // [Tmax*K]
@@ -181,25 +183,35 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(const __grid_constant_
   __syncthreads();
   if (p.S && threadIdx.x == 0) p.group_count[p.El] = T;
   __syncthreads();
-  int base_rows = 0, base_tiles = 0;
+  int base_rows = 0, base_tiles = 0, base_tiles2 = 0;
   for (int g0 = 0; g0 < p.G; g0 += blockDim.x) {
     const int g = g0 + threadIdx.x;
     const int cnt = g < p.G ? p.group_count[g] : 0;
-    int tot_rows, tot_tiles;
+    int tot_rows, tot_tiles, tot_tiles2;
     const int ex_rows = block_exclusive_scan(cnt, s_warp, &tot_rows);
     const int ex_tiles = block_exclusive_scan((cnt + kTileM - 1) / kTileM, s_warp, &tot_tiles);
+    const int ex_tiles2 =
+        block_exclusive_scan((cnt + 2 * kTileM - 1) / (2 * kTileM), s_warp, &tot_tiles2);
     if (g < p.G) {
       p.group_off[g] = base_rows + ex_rows;
       p.mtile_off[g] = base_tiles + ex_tiles;
+      if (p.mtile2_off) p.mtile2_off[g] = base_tiles2 + ex_tiles2;
     }
     base_rows += tot_rows;
     base_tiles += tot_tiles;
+    base_tiles2 += tot_tiles2;
   }
   if (threadIdx.x == 0) {
     p.group_off[p.G] = base_rows;
     p.mtile_off[p.G] = base_tiles;
+    if (p.mtile2_off) p.mtile2_off[p.G] = base_tiles2;
     p.info[1] = base_rows;
     p.info[2] = base_tiles;
+    // CTA-pair tiles cut the operand traffic per MMA, but every K block then needs a
+    // handshake between the two SMs (partial ready / partial drained) and the two TMEM
+    // buffers leave only one K block of slack for it: on the measured workloads the pair
+    // tiling ran about 2x slower, so it is used only when requested
+    p.info[3] = p.tiling == 2 ? 2 : 1;
   }
 }
 

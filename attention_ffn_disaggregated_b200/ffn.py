@@ -77,6 +77,8 @@ def lib() -> ctypes.CDLL:
         "afd_ffn_get_kernel_times": (c_int32, [P, POINTER(c_float)]),
         "afd_ffn_set_wait_limit": (c_int32, [P, c_int64]),
         "afd_ffn_inject_stall": (c_int32, [P, c_int32]),
+        "afd_ffn_set_tiling": (c_int32, [P, c_int32]),
+        "afd_ffn_get_tiling": (c_int32, [P, P, POINTER(c_int32)]),
         "afd_ffn_kernels_per_layer": (c_int32, []),
         "afd_ffn_route_noalloc": (c_int32, [POINTER(Config), POINTER(SlabDesc), P, P, P, P, P, P, P, P,
                                             P, P]),
@@ -212,6 +214,20 @@ class FfnLayer:
         rc = lib().afd_ffn_set_wait_limit(self.plan, int(ns))
         if rc != AFD_OK:
             raise AfdError(rc, "afd_ffn_set_wait_limit")
+
+    def set_tiling(self, tiling: int):
+        """0: chosen per call on the device; 1: single-CTA tiles; 2: CTA-pair tiles."""
+        rc = lib().afd_ffn_set_tiling(self.plan, int(tiling))
+        if rc != AFD_OK:
+            raise AfdError(rc, "afd_ffn_set_tiling")
+
+    def tiling(self, stream=None) -> int:
+        """Tiling (1 or 2) the last layer call used."""
+        t = c_int32(0)
+        rc = lib().afd_ffn_get_tiling(self.plan, c_void_p(_stream_handle(stream)), ctypes.byref(t))
+        if rc != AFD_OK:
+            raise AfdError(rc, "afd_ffn_get_tiling")
+        return t.value
 
     def inject_stall(self, enable: bool = True):
         lib().afd_ffn_inject_stall(self.plan, 1 if enable else 0)

@@ -249,6 +249,7 @@ def main():
     if rc != 0:
         raise RuntimeError(f"layer status {rc} word {word:#x}")
     rt = layer.routing()
+    tiling = layer.tiling()
     bytes_alg, flops_alg, R, active = workload_bytes_flops(inp, rt["counts"])
 
     layer.set_timing(True)
@@ -356,6 +357,8 @@ def main():
                        "intermediate": I, "local_experts": inp.shape.num_local_experts,
                        "shared_expert": inp.shape.has_shared_expert, "top_k": inp.shape.top_k,
                        "routed_rows": R, "active_experts": active,
+                       "gemm_tiling": {1: "one CTA per 128x256 tile",
+                                       2: "CTA pairs on 256x256 tiles (cta_group::2)"}[tiling],
                        "l2": "flushed between steps (256 MiB write, untimed)",
                        "parallelism": f"replica x{world}"},
             "roofline": {"bound": "tensor", "kernel": dominant, "achieved": achieved,

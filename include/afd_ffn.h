@@ -78,7 +78,8 @@ typedef enum {
 #define AFD_MAX_GROUPS 1024 /* num_local_experts + has_shared_expert */
 #define AFD_QBLOCK 128      /* quantisation block edge */
 
-/* Device kernels of one layer call, in launch order (for afd_ffn_get_kernel_times). */
+/* Timed stages of one layer call, in launch order (for afd_ffn_get_kernel_times); the
+ * two GEMM stages each cover the launches of both tilings. */
 #define AFD_KERNEL_ROUTE_COUNT 0
 #define AFD_KERNEL_ROUTE_SCAN 1
 #define AFD_KERNEL_ROUTE_SCATTER 2
@@ -199,6 +200,17 @@ AFD_API afd_status_t afd_ffn_set_timing(afd_ffn_plan_t plan, int32_t enable);
 AFD_API afd_status_t afd_ffn_get_kernel_times(afd_ffn_plan_t plan, float* ms);
 
 /*
+ * Tiling of the two grouped GEMMs. 0 (default) or 1: one CTA per 128-row x 256-column
+ * tile; 2: CTA pairs on 256-row tiles (cta_group::2 MMAs, less operand traffic per MMA,
+ * but a per-K-block handshake between the two SMs that measured about 2x slower).
+ * Results are the same within rounding; tiling 2 exists for tests and measurements.
+ */
+AFD_API afd_status_t afd_ffn_set_tiling(afd_ffn_plan_t plan, int32_t tiling);
+
+/* Synchronise `stream` and report the tiling (1 or 2) the last layer call used. */
+AFD_API afd_status_t afd_ffn_get_tiling(afd_ffn_plan_t plan, afd_stream_t stream, int32_t* tiling);
+
+/*
  * Limit, in nanoseconds, of every bounded device wait (default 1e9). Used by tests to
  * make an injected stall expire quickly.
  */
@@ -248,7 +260,7 @@ AFD_API afd_status_t afd_ffn_route_noalloc(const afd_ffn_config_t* cfg, const af
                                            float* d_row_weight, int32_t* d_pos, int32_t* d_status,
                                            afd_stream_t stream);
 
-/* Number of this library's kernels one afd_ffn_layer call launches. */
+/* Number of this library's kernel launches one afd_ffn_layer call makes. */
 AFD_API int32_t afd_ffn_kernels_per_layer(void);
 
 /* Human-readable name of a status code. */

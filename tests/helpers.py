@@ -11,8 +11,9 @@ from oracle import fp8 as ofp8
 TOL_ROW_RMS = 2e-2
 
 
-def run_cuda_layer(inp, calls: int = 1, layer=None):
-    """Plan (unless given), run `calls` times on the current stream, return outputs/routing."""
+def run_cuda_layer(inp, calls: int = 1, layer=None, tiling: int = 0):
+    """Plan (unless given), run `calls` times on the current stream, return outputs/routing.
+    tiling: 0 = chosen on the device per call, 1 = single-CTA tiles, 2 = CTA-pair tiles."""
     import torch
     from attention_ffn_disaggregated_b200 import FfnLayer
     from attention_ffn_disaggregated_b200.device import (gather_outputs, to_device_counts,
@@ -21,6 +22,7 @@ def run_cuda_layer(inp, calls: int = 1, layer=None):
     if own:
         w = to_device_weights(inp)
         layer = FfnLayer(inp.shape, len(inp.slabs), inp.capacity, *w)
+    layer.set_tiling(tiling)
     slabs = to_device_slabs(inp)
     counts = to_device_counts(inp)
     outs = []
@@ -33,7 +35,7 @@ def run_cuda_layer(inp, calls: int = 1, layer=None):
     rc, word = layer.status()
     rt = layer.routing()
     res = {"outs": outs, "status_rc": rc, "status_word": word, "routing": rt, "layer": layer,
-           "slabs": slabs}
+           "slabs": slabs, "tiling": layer.tiling()}
     return res
 
 

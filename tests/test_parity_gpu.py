@@ -15,8 +15,8 @@ from tests.helpers import compare_outputs, compare_routing, run_cuda_layer
 pytestmark = pytest.mark.gpu
 
 
-def _full_check(inp, calls=1):
-    res = run_cuda_layer(inp, calls=calls)
+def _full_check(inp, calls=1, tiling=0):
+    res = run_cuda_layer(inp, calls=calls, tiling=tiling)
     ref = offn.ffn_layer(inp)
     compare_routing(res["routing"], ref["routing"])
     worst = [compare_outputs(o, ref["out"]) for o in res["outs"]]
@@ -38,6 +38,20 @@ def test_tiny_config():
 def test_random_shapes_several_tiles(seed, shape, counts, cap, zipf):
     inp = W.make_custom_inputs(shape, counts, cap, seed=seed, zipf_s=zipf)
     res, _, _ = _full_check(inp)
+    assert res["status_rc"] == 0
+
+
+@pytest.mark.parametrize("tiling", [1, 2])
+@pytest.mark.parametrize("seed,shape,counts,cap", [
+    # experts of a few hundred rows: pair tiles whose second CTA is partly or fully empty
+    (21, W.LayerShape(512, 256, 4, 0, 4, 1, 2), [300, 217, 0, 65], 300),
+    (22, W.LayerShape(768, 384, 6, 0, 6, 0, 3), [511, 2], 511),
+    (23, W.LayerShape(1024, 256, 16, 4, 6, 1, 4), [1, 0, 130], 130),
+])
+def test_both_tilings(tiling, seed, shape, counts, cap):
+    inp = W.make_custom_inputs(shape, counts, cap, seed=seed, zipf_s=1.0)
+    res, _, _ = _full_check(inp, calls=2, tiling=tiling)
+    assert res["tiling"] == tiling
     assert res["status_rc"] == 0
 
 
@@ -130,10 +144,10 @@ def test_timeout_injection_reports_status_and_recovers():
 
 # ------------------------------------------------------------------ full-size workloads
 
-def _sampled_check(name, n_sample=40):
+def _sampled_check(name, n_sample=40, tiling=0):
     wl = W.CONFIGS[name]
     inp = W.make_inputs(wl)
-    res = run_cuda_layer(inp)
+    res = run_cuda_layer(inp, tiling=tiling)
     assert res["status_rc"] == 0
     ort = offn.route_inputs(inp)
     compare_routing(res["routing"], ort)
@@ -144,7 +158,8 @@ def _sampled_check(name, n_sample=40):
     return compare_outputs(res["outs"][0], ref["out"], tokens=toks)
 
 
-@pytest.mark.parametrize("name", ["qwen3_235b_t2048", "deepseek_v3_share_t4096",
-                                  "qwen3_235b_spec_q4_t8192"])
-def test_full_size_sampled(name):
-    _sampled_check(name)
+@pytest.mark.parametrize("name,tiling", [("qwen3_235b_t2048", 0), ("deepseek_v3_share_t4096", 0),
+                                         ("deepseek_v3_share_t4096", 2),
+                                         ("qwen3_235b_spec_q4_t8192", 0)])
+def test_full_size_sampled(name, tiling):
+    _sampled_check(name, tiling=tiling)
