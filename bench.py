@@ -44,6 +44,12 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-tokens", type=int, default=64)
+    ap.add_argument("--graph", action="store_true",
+                    help="time replays of the layer captured in a CUDA graph")
+    ap.add_argument("--sweep", action="store_true",
+                    help="batch / fan-in sweep at the DeepSeek-V3 share shape: one line per cell")
+    ap.add_argument("--sweep-filter", default="",
+                    help="only sweep cells whose name contains this string")
     return ap.parse_args()
 
 
@@ -208,10 +214,88 @@ def run_reference(args):
     return 0
 
 
+def time_layer(layer, slabs, counts, flush, steps, warmup, graph=False):
+    """Device time of `steps` layer calls (ms each), L2 flushed before every call."""
+    import torch
+    stream = torch.cuda.current_stream()
+    run = lambda: layer(slabs, counts)
+    g = None
+    if graph:
+        layer.set_timing(False)          # no per-kernel events inside the captured graph
+        side = torch.cuda.Stream()
+        with torch.cuda.stream(side):
+            layer(slabs, counts)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=side):
+            layer(slabs, counts)
+        run = g.replay
+    for _ in range(warmup):
+        flush.zero_()
+        run()
+    torch.cuda.synchronize()
+    out = []
+    for _ in range(steps):
+        flush.zero_()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        run()
+        e1.record(stream)
+        e1.synchronize()
+        out.append(e0.elapsed_time(e1))
+    del g
+    if graph:
+        layer.set_timing(True)
+    return out
+
+
+def run_sweep(args):
+    """FFN-stage time T_e against batch T and fan-in M (the per-layer term of the overlap
+    model), at the DeepSeek-V3 share shape, uniform and Zipf(1.2) routing."""
+    import torch
+    from attention_ffn_disaggregated_b200 import FfnLayer
+    from attention_ffn_disaggregated_b200.device import (to_device_counts, to_device_slabs,
+                                                          to_device_weights)
+    cells = [w for w in W.sweep_workloads() if args.sweep_filter in w.name]
+    weights = W.make_weights(W.DEEPSEEK_V3_SHARE, torch.Generator().manual_seed(4))
+    hbm, bf16, _, _ = measured_peaks()
+    fp8_peak = 2.0 * bf16
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    dev_w = None
+    for wl in cells:
+        inp = W.make_inputs(wl, weights=weights)
+        if dev_w is None:
+            dev_w = to_device_weights(inp)
+        layer = FfnLayer(inp.shape, len(inp.slabs), inp.capacity, *dev_w)
+        slabs = to_device_slabs(inp, y_fill=0.0)
+        counts = to_device_counts(inp)
+        layer(slabs, counts)
+        rc, word = layer.status()
+        rt = layer.routing()
+        bytes_alg, flops_alg, R, active = workload_bytes_flops(inp, rt["counts"])
+        ms = time_layer(layer, slabs, counts, flush, args.steps, args.warmup, graph=args.graph)
+        t = float(np.median(ms))
+        T = int(np.sum(inp.counts))
+        t_roof = max(bytes_alg / (hbm * 1e9), flops_alg / (fp8_peak * 1e12)) * 1e3
+        print(json.dumps({"cell": wl.name, "tokens": T, "slabs": wl.num_slabs,
+                          "routing": "uniform" if wl.zipf_s is None else f"zipf{wl.zipf_s}",
+                          "routed_rows": R, "active_experts": active, "ms": t,
+                          "tokens_per_s": T / (t * 1e-3), "t_roof_ms": t_roof,
+                          "roofline_frac": t_roof / t,
+                          "bound": "tensor" if flops_alg / (fp8_peak * 1e12) >= bytes_alg / (hbm * 1e9) else "hbm",
+                          "status": rc, "graph": bool(args.graph)}), flush=True)
+        layer.close()
+        del layer, slabs
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
+    if args.sweep:
+        return run_sweep(args)
 
     import torch
     import torch.distributed as dist
@@ -265,15 +349,27 @@ def main():
                           "gemm13_swiglu", "gemm2_combine", "combine_finalize")}
     step_ms = []
     with ClockSampler(local) as clk:
-        for _ in range(args.steps):
+        if args.graph:
+            # the whole layer replayed from a CUDA graph; per-kernel times come from a
+            # separate pass of directly launched calls below
+            step_ms = time_layer(layer, slabs, counts, flush, args.steps, 0, graph=True)
+        else:
+            for _ in range(args.steps):
+                flush.zero_()
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                layer(slabs, counts)
+                e1.record(stream)
+                e1.synchronize()
+                step_ms.append(e0.elapsed_time(e1))
+                for k, v in layer.kernel_times().items():
+                    kt[k].append(v)
+    if args.graph:
+        for _ in range(min(args.steps, 5)):
             flush.zero_()
-            e0 = torch.cuda.Event(enable_timing=True)
-            e1 = torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
             layer(slabs, counts)
-            e1.record(stream)
-            e1.synchronize()
-            step_ms.append(e0.elapsed_time(e1))
+            torch.cuda.synchronize()
             for k, v in layer.kernel_times().items():
                 kt[k].append(v)
     torch.cuda.synchronize()
@@ -360,6 +456,7 @@ def main():
                        "gemm_tiling": {1: "one CTA per 128x256 tile",
                                        2: "CTA pairs on 256x256 tiles (cta_group::2)"}[tiling],
                        "l2": "flushed between steps (256 MiB write, untimed)",
+                       "launch": "CUDA graph replay" if args.graph else "direct launches",
                        "parallelism": f"replica x{world}"},
             "roofline": {"bound": "tensor", "kernel": dominant, "achieved": achieved,
                          "peak": fp8_peak, "unit": "TFLOP/s", "frac": achieved / fp8_peak,
