@@ -428,7 +428,7 @@ afd_status_t afd_ffn_layer(afd_ffn_plan_t P, const afd_slab_t* slabs, const int3
   if (tm) cudaEventRecord(P->ev[2], stream);
   route_scatter_kernel<<<P->num_chunks, kRouteThreads, P->scatter_smem, stream>>>(rp, tab);
   if (tm) cudaEventRecord(P->ev[3], stream);
-  gather_rows_kernel<<<P->num_sms * 4, kRouteThreads, 0, stream>>>(rp, tab);
+  gather_rows_kernel<<<P->num_sms * 8, kRouteThreads, 0, stream>>>(rp, tab);
   if (tm) cudaEventRecord(P->ev[4], stream);
   // both tilings are launched; the one the routing scan did not choose exits at entry
   const int grid1 = P->num_sms, grid2 = P->num_sms & ~1;

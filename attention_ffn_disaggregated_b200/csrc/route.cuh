@@ -326,13 +326,12 @@ __global__ void __launch_bounds__(kRouteThreads) gather_rows_kernel(
     uint4* __restrict__ dst = reinterpret_cast<uint4*>(p.a_perm + static_cast<size_t>(r) * p.H);
     const int n16 = p.H / 16;             // H is a multiple of 256: n16 a multiple of 16
     int i = lane;
-    for (; i + 96 < n16; i += 128) {      // four 16-byte loads in flight per lane
-      const uint4 a = __ldg(src + i), b = __ldg(src + i + 32), c = __ldg(src + i + 64),
-                  d = __ldg(src + i + 96);
-      dst[i] = a;
-      dst[i + 32] = b;
-      dst[i + 64] = c;
-      dst[i + 96] = d;
+    for (; i + 7 * 32 < n16; i += 8 * 32) {   // eight 16-byte loads in flight per lane
+      uint4 v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = __ldg(src + i + 32 * j);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) dst[i + 32 * j] = v[j];
     }
     for (; i < n16; i += 32) dst[i] = __ldg(src + i);
     const float* ssrc = slabs.xs[m] + static_cast<size_t>(t) * KB;
