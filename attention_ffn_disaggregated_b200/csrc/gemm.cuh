@@ -95,7 +95,8 @@ struct GemmParams {
   int inject_stall;
 };
 
-struct GemmSmem {
+// 16-byte multiple: the combine staging that follows it is accessed as float4
+struct alignas(16) GemmSmem {
   uint64_t full[kMaxStages];
   uint64_t empty[kMaxStages];
   uint64_t tfull[2];
@@ -108,6 +109,7 @@ struct GemmSmem {
 };
 
 constexpr size_t kGemmSmemTiles = static_cast<size_t>(192) * 1024;   // both tilings
+static_assert(sizeof(GemmSmem) % 16 == 0, "staging after GemmSmem must stay 16-byte aligned");
 static_assert(Tiling<1>::kStages * Tiling<1>::kStageBytes == kGemmSmemTiles, "tiling size");
 static_assert(Tiling<2>::kStages * Tiling<2>::kStageBytes == kGemmSmemTiles, "tiling size");
 constexpr size_t kStgBytes = static_cast<size_t>(kEpiWarps) * 32 * kStgStride * sizeof(float);
