@@ -41,7 +41,7 @@ constexpr int kBK = 128;
 constexpr int kGemmThreads = 384;
 constexpr int kEpiWarps = 8;
 constexpr uint32_t kABytes = kTileM * kBK;   // 16 KiB: 128 rows of one K block
-constexpr int kStgStride = 20;               // floats per staging row (16 + 4 pad)
+constexpr int kStgStride = 36;               // floats per staging row (32 + 4 pad)
 constexpr uint32_t kTmemCols = 512;          // two 256-column fp32 partial buffers
 constexpr int kMaxStages = 6;
 // Register split: the block launches with kLaunchRegs per thread; warpgroup 0 (TMA, MMA,
@@ -112,7 +112,7 @@ constexpr size_t kGemmSmemTiles = static_cast<size_t>(192) * 1024;   // both til
 static_assert(sizeof(GemmSmem) % 16 == 0, "staging after GemmSmem must stay 16-byte aligned");
 static_assert(Tiling<1>::kStages * Tiling<1>::kStageBytes == kGemmSmemTiles, "tiling size");
 static_assert(Tiling<2>::kStages * Tiling<2>::kStageBytes == kGemmSmemTiles, "tiling size");
-constexpr size_t kStgBytes = static_cast<size_t>(kEpiWarps) * 32 * kStgStride * sizeof(float);
+constexpr size_t kStgBytes = static_cast<size_t>(kEpiWarps) * 16 * kStgStride * sizeof(float);
 
 __host__ __device__ constexpr size_t gemm_smem_bytes(int epi) {
   return 1024 + kGemmSmemTiles + sizeof(GemmSmem) + (epi == EPI_COMBINE ? kStgBytes : 0);
@@ -453,35 +453,42 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       } else {
         // weighted combine: fp32 reductions into the token accumulator (kept in L2 with
         // an evict-last hint), staged through shared memory so that each reduction covers
-        // 128 contiguous bytes of one row; combine_finalize_kernel turns the sums into bf16
+        // 128 contiguous bytes of a row; combine_finalize_kernel turns the sums into bf16
         int g = -1;
         float wgt = 0.f;
         if (valid) {
           g = p.row_token[grow];
           wgt = p.row_w[grow];
         }
-        float* sw = stg + ew * 32 * kStgStride;
+        // the 32 rows go through the staging in two halves of 16; a reduction instruction
+        // then covers 4 rows x 128 contiguous bytes (8 lanes per row)
+        float* sw = stg + ew * 16 * kStgStride;
         const int col0 = c.nt * kBN + half * 128;
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
+        for (int ch = 0; ch < 4; ++ch) {          // 32 columns per chunk
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const float2 a = acc[8 * ch + 2 * j], bb = acc[8 * ch + 2 * j + 1];
-            *reinterpret_cast<float4*>(sw + lane * kStgStride + 4 * j) =
-                make_float4(a.x * wgt, a.y * wgt, bb.x * wgt, bb.y * wgt);
-          }
-          __syncwarp();
+          for (int hr = 0; hr < 2; ++hr) {
+            if ((lane >> 4) == hr) {
 #pragma unroll
-          for (int r4 = 0; r4 < 4; ++r4) {
-            const int rr = r4 * 8 + (lane >> 2);
-            const int cc = (lane & 3) * 4;
-            const int gg = __shfl_sync(0xffffffffu, g, rr);
-            const float4 v = *reinterpret_cast<const float4*>(sw + rr * kStgStride + cc);
-            if (gg >= 0)
-              red_add_v4_hint(p.acc + static_cast<size_t>(gg) * p.H + col0 + 16 * ch + cc, v.x,
-                              v.y, v.z, v.w, pol_acc);
+              for (int j = 0; j < 8; ++j) {
+                const float2 a = acc[16 * ch + 2 * j], bb = acc[16 * ch + 2 * j + 1];
+                *reinterpret_cast<float4*>(sw + (lane & 15) * kStgStride + 4 * j) =
+                    make_float4(a.x * wgt, a.y * wgt, bb.x * wgt, bb.y * wgt);
+              }
+            }
+            __syncwarp();
+#pragma unroll
+            for (int r4 = 0; r4 < 4; ++r4) {
+              const int rl = r4 * 4 + (lane >> 3);
+              const int cc = (lane & 7) * 4;
+              const int gg = __shfl_sync(0xffffffffu, g, 16 * hr + rl);
+              const float4 v = *reinterpret_cast<const float4*>(sw + rl * kStgStride + cc);
+              if (gg >= 0)
+                red_add_v4_hint(p.acc + static_cast<size_t>(gg) * p.H + col0 + 32 * ch + cc, v.x,
+                                v.y, v.z, v.w, pol_acc);
+            }
+            __syncwarp();
           }
-          __syncwarp();
         }
       }
     }
