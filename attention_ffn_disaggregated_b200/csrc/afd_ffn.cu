@@ -62,6 +62,10 @@ struct afd_ffn_plan_s {
   uint8_t *a_perm, *hq;
   int* status;
   CUtensorMap tm_a13, tm_w13, tm_a2, tm_w2;
+  // tiling 3 (W13 rows gathered from the slabs): one map per slab, re-encoded when a slab's
+  // row pointer changes between calls
+  AMaps<true> slab_maps;
+  const void* slab_x[AFD_MAX_SLABS] = {};
   bool timing = false, ev_valid = false;
   cudaEvent_t ev[AFD_NUM_KERNELS + 1] = {};
   unsigned long long wait_limit_ns = 1000000000ull;
@@ -84,8 +88,8 @@ const char* afd_status_string(afd_status_t s) {
   return "unknown";
 }
 
-// route count, scan, scatter, gather, W13 (two tilings), W2 (two tilings), finalize
-int32_t afd_ffn_kernels_per_layer(void) { return 9; }
+// route count, scan, scatter, gather, W13, W2, finalize
+int32_t afd_ffn_kernels_per_layer(void) { return 7; }
 
 afd_status_t afd_ffn_check_config(const afd_ffn_config_t* c) {
   if (!c) return AFD_ERR_INVALID_ARGUMENT;
@@ -126,6 +130,19 @@ static afd_status_t encode_2d(EncodeTiledFn enc, CUtensorMap* m, void* base, uin
   return r == CUDA_SUCCESS ? AFD_OK : AFD_ERR_CUDA;
 }
 
+// A slab's FP8 rows [cap][H] for tile::gather4: box {128 columns, 1 row}.
+static afd_status_t encode_slab(EncodeTiledFn enc, CUtensorMap* m, const void* x, uint64_t H,
+                                uint64_t cap) {
+  cuuint64_t dims[2] = {H, cap};
+  cuuint64_t strides[1] = {H};
+  cuuint32_t box[2] = {128, 1};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(x), dims, strides, box, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? AFD_OK : AFD_ERR_CUDA;
+}
+
 static afd_status_t encode_3d(EncodeTiledFn enc, CUtensorMap* m, const void* base, uint64_t inner,
                               uint64_t rows, uint64_t experts, uint32_t box_rows) {
   cuuint64_t dims[3] = {inner, rows, experts};
@@ -160,10 +177,11 @@ afd_status_t afd_ffn_plan(const afd_ffn_config_t* cfg, const afd_ffn_weights_t* 
   // The GEMM kernels split the block's registers between warpgroups with setmaxnreg; that
   // is only safe when the block is launched with exactly the budget the split assumes.
   {
-    const void* fns[4] = {reinterpret_cast<const void*>(grouped_gemm_kernel<EPI_SWIGLU, 1>),
-                          reinterpret_cast<const void*>(grouped_gemm_kernel<EPI_SWIGLU, 2>),
-                          reinterpret_cast<const void*>(grouped_gemm_kernel<EPI_COMBINE, 1>),
-                          reinterpret_cast<const void*>(grouped_gemm_kernel<EPI_COMBINE, 2>)};
+    const void* fns[5] = {reinterpret_cast<const void*>(grouped_gemm_kernel<EPI_SWIGLU, 1, false>),
+                          reinterpret_cast<const void*>(grouped_gemm_kernel<EPI_SWIGLU, 1, true>),
+                          reinterpret_cast<const void*>(grouped_gemm_kernel<EPI_SWIGLU, 2, false>),
+                          reinterpret_cast<const void*>(grouped_gemm_kernel<EPI_COMBINE, 1, false>),
+                          reinterpret_cast<const void*>(grouped_gemm_kernel<EPI_COMBINE, 2, false>)};
     for (const void* fn : fns) {
       cudaFuncAttributes fa;
       if (cudaFuncGetAttributes(&fa, fn) != cudaSuccess) return AFD_ERR_CUDA;
@@ -261,13 +279,15 @@ afd_status_t afd_ffn_plan(const afd_ffn_config_t* cfg, const afd_ffn_weights_t* 
     return st;
   }
   P->scatter_smem = sizeof(int32_t) * (static_cast<size_t>(kRouteWarps) * El1 + kRouteWarps * 32 * K);
-  if (cudaFuncSetAttribute(grouped_gemm_kernel<EPI_SWIGLU, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (cudaFuncSetAttribute(grouped_gemm_kernel<EPI_SWIGLU, 1, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(gemm_smem_bytes(EPI_SWIGLU))) != cudaSuccess ||
-      cudaFuncSetAttribute(grouped_gemm_kernel<EPI_SWIGLU, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      cudaFuncSetAttribute(grouped_gemm_kernel<EPI_SWIGLU, 1, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(gemm_smem_bytes(EPI_SWIGLU))) != cudaSuccess ||
-      cudaFuncSetAttribute(grouped_gemm_kernel<EPI_COMBINE, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      cudaFuncSetAttribute(grouped_gemm_kernel<EPI_SWIGLU, 2, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(gemm_smem_bytes(EPI_SWIGLU))) != cudaSuccess ||
+      cudaFuncSetAttribute(grouped_gemm_kernel<EPI_COMBINE, 1, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(gemm_smem_bytes(EPI_COMBINE))) != cudaSuccess ||
-      cudaFuncSetAttribute(grouped_gemm_kernel<EPI_COMBINE, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      cudaFuncSetAttribute(grouped_gemm_kernel<EPI_COMBINE, 2, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(gemm_smem_bytes(EPI_COMBINE))) != cudaSuccess ||
       // the limit is a per-function setting shared by every plan: set the largest any
       // configuration can need, so that a later plan never lowers an earlier plan's limit
@@ -305,7 +325,8 @@ afd_status_t afd_ffn_get_info(afd_ffn_plan_t P, afd_ffn_plan_info_t* info) {
 }
 
 // Launch a CTA-pair kernel: clusters of two consecutive CTAs.
-static cudaError_t launch_pair(void (*kernel)(GemmParams, CUtensorMap, CUtensorMap, YTable), int grid,
+static cudaError_t launch_pair(void (*kernel)(GemmParams, CUtensorMap, CUtensorMap, YTable, AMaps<false>),
+                               int grid,
                                size_t smem, cudaStream_t stream, const GemmParams& gp,
                                const CUtensorMap& ta, const CUtensorMap& tb, const YTable& ytab) {
   cudaLaunchConfig_t cfg = {};
@@ -320,7 +341,7 @@ static cudaError_t launch_pair(void (*kernel)(GemmParams, CUtensorMap, CUtensorM
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kernel, gp, ta, tb, ytab);
+  return cudaLaunchKernelEx(&cfg, kernel, gp, ta, tb, ytab, AMaps<false>{0});
 }
 
 static void fill_route_params(afd_ffn_plan_t P, const int32_t* d_counts, RouteParams& rp) {
@@ -370,6 +391,8 @@ static void fill_gemm_params(afd_ffn_plan_t P, int epi, GemmParams& gp) {
   gp.H = c.hidden;
   gp.status = P->status;
   gp.wait_limit_ns = P->wait_limit_ns;
+  gp.row_token = P->row_token;
+  gp.tok_mt = P->tok_mt;
   if (epi == EPI_SWIGLU) {
     gp.n_tiles = c.intermediate / 128;
     gp.num_kb = c.hidden / 128;
@@ -385,7 +408,6 @@ static void fill_gemm_params(afd_ffn_plan_t P, int epi, GemmParams& gp) {
     gp.sa_t = P->sh_t;
     gp.w_scale = P->w.w2_scale;
     gp.ws_rows = c.hidden / 128;
-    gp.row_token = P->row_token;
     gp.row_w = P->row_w;
     gp.acc = P->acc;
   }
@@ -413,6 +435,22 @@ afd_status_t afd_ffn_layer(afd_ffn_plan_t P, const afd_slab_t* slabs, const int3
     tab.y[m] = static_cast<__nv_bfloat16*>(s.y);
     ytab.y[m] = static_cast<__nv_bfloat16*>(s.y);
   }
+  // tilings 1 (default) and 2 read an expert-ordered copy of the rows made by the gather
+  // stage; tiling 3 gathers them from the slabs inside the W13 kernel (tile::gather4)
+  const int tiling = P->tiling == 0 ? 1 : P->tiling;
+  const bool pair = tiling == 2, slab_gather = tiling == 3;
+  if (slab_gather) {
+    EncodeTiledFn enc = get_encode_fn();
+    if (!enc) return AFD_ERR_CUDA;
+    for (int m = 0; m < c.num_slabs; ++m) {
+      if (P->slab_x[m] == slabs[m].x) continue;
+      if (encode_slab(enc, &P->slab_maps.m[m], slabs[m].x, c.hidden, c.slab_capacity) != AFD_OK) {
+        P->slab_x[m] = nullptr;
+        return AFD_ERR_CUDA;
+      }
+      P->slab_x[m] = slabs[m].x;
+    }
+  }
   RouteParams rp;
   fill_route_params(P, d_counts, rp);
   GemmParams g13, g2;
@@ -428,21 +466,28 @@ afd_status_t afd_ffn_layer(afd_ffn_plan_t P, const afd_slab_t* slabs, const int3
   if (tm) cudaEventRecord(P->ev[2], stream);
   route_scatter_kernel<<<P->num_chunks, kRouteThreads, P->scatter_smem, stream>>>(rp, tab);
   if (tm) cudaEventRecord(P->ev[3], stream);
-  gather_rows_kernel<<<P->num_sms * 8, kRouteThreads, 0, stream>>>(rp, tab);
+  if (slab_gather) gather_scales_kernel<<<P->num_sms * 4, kRouteThreads, 0, stream>>>(rp, tab);
+  else gather_rows_kernel<<<P->num_sms * 8, kRouteThreads, 0, stream>>>(rp, tab);
   if (tm) cudaEventRecord(P->ev[4], stream);
-  // both tilings are launched; the one the routing scan did not choose exits at entry
   const int grid1 = P->num_sms, grid2 = P->num_sms & ~1;
-  grouped_gemm_kernel<EPI_SWIGLU, 1><<<grid1, kGemmThreads, gemm_smem_bytes(EPI_SWIGLU), stream>>>(
-      g13, P->tm_a13, P->tm_w13, ytab);
-  if (launch_pair(grouped_gemm_kernel<EPI_SWIGLU, 2>, grid2, gemm_smem_bytes(EPI_SWIGLU), stream, g13,
-                  P->tm_a13, P->tm_w13, ytab) != cudaSuccess)
+  if (slab_gather) {
+    grouped_gemm_kernel<EPI_SWIGLU, 1, true><<<grid1, kGemmThreads, gemm_smem_bytes(EPI_SWIGLU), stream>>>(
+        g13, P->tm_a13, P->tm_w13, ytab, P->slab_maps);
+  } else if (!pair) {
+    grouped_gemm_kernel<EPI_SWIGLU, 1, false><<<grid1, kGemmThreads, gemm_smem_bytes(EPI_SWIGLU), stream>>>(
+        g13, P->tm_a13, P->tm_w13, ytab, AMaps<false>{0});
+  } else if (launch_pair(grouped_gemm_kernel<EPI_SWIGLU, 2, false>, grid2, gemm_smem_bytes(EPI_SWIGLU),
+                         stream, g13, P->tm_a13, P->tm_w13, ytab) != cudaSuccess) {
     return AFD_ERR_CUDA;
+  }
   if (tm) cudaEventRecord(P->ev[5], stream);
-  grouped_gemm_kernel<EPI_COMBINE, 1><<<grid1, kGemmThreads, gemm_smem_bytes(EPI_COMBINE), stream>>>(
-      g2, P->tm_a2, P->tm_w2, ytab);
-  if (launch_pair(grouped_gemm_kernel<EPI_COMBINE, 2>, grid2, gemm_smem_bytes(EPI_COMBINE), stream, g2,
-                  P->tm_a2, P->tm_w2, ytab) != cudaSuccess)
+  if (!pair) {
+    grouped_gemm_kernel<EPI_COMBINE, 1, false><<<grid1, kGemmThreads, gemm_smem_bytes(EPI_COMBINE), stream>>>(
+        g2, P->tm_a2, P->tm_w2, ytab, AMaps<false>{0});
+  } else if (launch_pair(grouped_gemm_kernel<EPI_COMBINE, 2, false>, grid2, gemm_smem_bytes(EPI_COMBINE),
+                         stream, g2, P->tm_a2, P->tm_w2, ytab) != cudaSuccess) {
     return AFD_ERR_CUDA;
+  }
   if (tm) cudaEventRecord(P->ev[6], stream);
   combine_finalize_kernel<<<P->num_sms * 4, 256, 0, stream>>>(P->info, P->tok_mt, P->acc, c.hidden, ytab);
   if (tm) cudaEventRecord(P->ev[7], stream);
@@ -535,7 +580,7 @@ afd_status_t afd_ffn_set_wait_limit(afd_ffn_plan_t P, int64_t limit_ns) {
 }
 
 afd_status_t afd_ffn_set_tiling(afd_ffn_plan_t P, int32_t tiling) {
-  if (!P || tiling < 0 || tiling > 2) return AFD_ERR_INVALID_ARGUMENT;
+  if (!P || tiling < 0 || tiling > 3) return AFD_ERR_INVALID_ARGUMENT;
   P->tiling = tiling;
   return AFD_OK;
 }

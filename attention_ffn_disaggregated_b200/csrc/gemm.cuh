@@ -69,8 +69,24 @@ struct YTable {
   __nv_bfloat16* y[AFD_MAX_SLABS];
 };
 
+// W13 A operand straight from the slabs: one 2D map per slab over its FP8 rows, box one
+// row high ({128 columns, 1 row}) so that tile::gather4 can fetch four arbitrary rows.
+template <bool GATHER>
+struct AMaps {
+  CUtensorMap m[AFD_MAX_SLABS];
+};
+template <>
+struct AMaps<false> {
+  int unused;
+};
+template <bool GATHER>
+__device__ __forceinline__ const CUtensorMap* slab_map(const AMaps<GATHER>& a, int m) {
+  if constexpr (GATHER) return &a.m[m];
+  else return nullptr;
+}
+
 struct GemmParams {
-  const int32_t* info;        // [3] = tiling chosen for this call (1 or 2)
+  const int32_t* info;        // [0] tokens, [1] rows, [2] m-tiles of this call
   const int32_t* group_off;   // [G+1] first row of each group
   const int32_t* mtile_off;   // [G+1] first 128-row m-tile of each group
   const int32_t* mtile2_off;  // [G+1] first 256-row m-tile of each group
@@ -86,7 +102,9 @@ struct GemmParams {
   // SWIGLU epilogue outputs
   uint8_t* hq;                // [rpad][I]
   float* sh_t;                // [I/128][rpad]
-  // COMBINE epilogue inputs/outputs
+  // W13 from the slabs: row -> token -> (slab << 24) | row in slab
+  const int32_t* tok_mt;
+  // COMBINE epilogue inputs/outputs (row_token also for the slab gather)
   const int32_t* row_token;
   const float* row_w;
   float* acc;                 // [Tmax][H] fp32, zero between calls
@@ -151,16 +169,18 @@ __device__ __forceinline__ TileCoord decode_tile(int tile, int n_tiles, const in
   return c;
 }
 
-template <int EPI, int PAIR>
+// GATHER (W13, single-CTA tiles only): the A tile's rows are fetched from the slabs
+// through `amaps` instead of from the expert-ordered copy behind `tm_a`.
+template <int EPI, int PAIR, bool GATHER>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ GemmParams p,
                         const __grid_constant__ CUtensorMap tm_a,
                         const __grid_constant__ CUtensorMap tm_b,
-                        const __grid_constant__ YTable ytab) {
+                        const __grid_constant__ YTable ytab,
+                        const __grid_constant__ AMaps<GATHER> amaps) {
+  static_assert(!GATHER || (EPI == EPI_SWIGLU && PAIR == 1), "slab gather: W13, single-CTA tiles");
   using TL = Tiling<PAIR>;
   constexpr int kStages = TL::kStages;
-  // only the tiling the routing stage chose for this call runs; the other launch exits
-  if (p.info[3] != PAIR) return;
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -212,7 +232,69 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp < 4) {
     // each role's code sits inside the branch that sets its register budget
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kProducerRegs));
-    if (warp == 0 && lane == 0) {
+    if (GATHER && warp == 0) {
+      // ------------------------------------------------- TMA producer, A rows from the slabs
+      // lane l fetches tile rows 4l..4l+3: one gather4 when the four share a slab, else one
+      // single-row copy each; rows past the group's end repeat the tile's first row
+      if (lane == 0) tma_prefetch_desc(&tm_b);
+      const uint64_t pol_a = policy_evict_last();
+      const uint64_t pol_b = policy_evict_last();
+      int it = 0;
+      bool ok = true;
+      int skipped = -1;
+      for (int tile = unit; ok && tile < total_tiles; tile += nunits) {
+        const TileCoord c = decode_tile<PAIR>(tile, p.n_tiles, S.mtile, p.G, p.group_off, rank);
+        const int brow0 = c.nt * 128;            // gate block
+        const int brow1 = p.I + c.nt * 128;      // up block
+        int rm[4], rt[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int r = 4 * lane + j;
+          const int mt = p.tok_mt[p.row_token[c.row0 + (r < c.rows ? r : 0)]];
+          rm[j] = mt >> 24;
+          rt[j] = mt & 0xFFFFFF;
+        }
+        const bool one_slab = rm[0] == rm[1] && rm[0] == rm[2] && rm[0] == rm[3];
+        for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
+          const int s = it % kStages;
+          const uint32_t ph = (it / kStages) & 1;
+          int got = 1;
+          if (lane == 0) got = mbar_wait(&S.empty[s], ph ^ 1, abort_flag, p.status, p.wait_limit_ns);
+          got = __shfl_sync(0xffffffffu, got, 0);
+          if (!got) {
+            ok = false;
+            break;
+          }
+          if (p.inject_stall && blockIdx.x == 0 && it == 0) {
+            skipped = it;       // test hook: never fill this stage
+            continue;
+          }
+          uint8_t* a = sA + s * kABytes + 4 * lane * kBK;
+          uint8_t* b = sB + s * TL::kBBytes;
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&S.full[s], TL::kTxBytes);
+            tma_load_3d(b, &tm_b, &S.full[s], kb * kBK, brow0, c.e, pol_b);
+            tma_load_3d(b + TL::kBBytes / 2, &tm_b, &S.full[s], kb * kBK, brow1, c.e, pol_b);
+          }
+          __syncwarp();
+          if (one_slab) {
+            tma_gather4(a, slab_map(amaps, rm[0]), &S.full[s], kb * kBK, rt[0], rt[1], rt[2], rt[3],
+                        pol_a);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              tma_load_2d(a + j * kBK, slab_map(amaps, rm[j]), &S.full[s], kb * kBK, rt[j], pol_a);
+          }
+        }
+      }
+      if (!ok && lane == 0) {
+        // wait (bounded) for copies that may still be landing on this CTA's barriers
+        for (int j = max(0, it - kStages); j < it; ++j) {
+          if (j == skipped) continue;
+          mbar_wait_drain(&S.full[j % kStages], (j / kStages) & 1, p.wait_limit_ns);
+        }
+      }
+    } else if (!GATHER && warp == 0 && lane == 0) {
       // ---------------------------------------------------------------- TMA producer
       tma_prefetch_desc(&tm_a);
       tma_prefetch_desc(&tm_b);

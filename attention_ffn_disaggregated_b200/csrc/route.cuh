@@ -40,7 +40,7 @@ struct RouteParams {
   int32_t* group_off;     // [G+1]
   int32_t* mtile_off;     // [G+1] 128-row m-tiles
   int32_t* mtile2_off;    // [G+1] 256-row m-tiles (CTA-pair tiling); may be null
-  int tiling;             // 0: choose per call from the counts; 1 or 2: forced
+  int tiling;             // as set on the plan: 0 (default, = 1), 1, 2 or 3
   int32_t* tok_mt;        // [Tmax] (slab << 24) | row
   int32_t* tok_need;      // [Tmax] contributions this GPU adds to the token
   int32_t* pos;           // [Tmax*K]
@@ -207,11 +207,8 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(const __grid_constant_
     if (p.mtile2_off) p.mtile2_off[p.G] = base_tiles2;
     p.info[1] = base_rows;
     p.info[2] = base_tiles;
-    // CTA-pair tiles cut the operand traffic per MMA, but every K block then needs a
-    // handshake between the two SMs (partial ready / partial drained) and the two TMEM
-    // buffers leave only one K block of slack for it: on the measured workloads the pair
-    // tiling ran about 2x slower, so it is used only when requested
-    p.info[3] = p.tiling == 2 ? 2 : 1;
+    // the tiling this call runs (the host launches only its kernels)
+    p.info[3] = p.tiling == 0 ? 1 : p.tiling;
   }
 }
 
@@ -336,6 +333,20 @@ __global__ void __launch_bounds__(kRouteThreads) gather_rows_kernel(
     for (; i < n16; i += 32) dst[i] = __ldg(src + i);
     const float* ssrc = slabs.xs[m] + static_cast<size_t>(t) * KB;
     for (int kb = lane; kb < KB; kb += 32) p.sa_t[static_cast<size_t>(kb) * p.rpad + r] = ssrc[kb];
+  }
+}
+
+// 4b. when the W13 GEMM fetches its A rows from the slabs itself, only the per-128 scales
+// move into expert order: one thread per row, so that each K block's 32 consecutive rows
+// are written with one coalesced store per warp.
+__global__ void __launch_bounds__(kRouteThreads) gather_scales_kernel(
+    const __grid_constant__ RouteParams p, const __grid_constant__ SlabTable slabs) {
+  const int R = p.info[1];
+  const int KB = p.H / AFD_QBLOCK;
+  for (int r = blockIdx.x * blockDim.x + threadIdx.x; r < R; r += gridDim.x * blockDim.x) {
+    const int mt = p.tok_mt[p.row_token[r]];
+    const float* __restrict__ src = slabs.xs[mt >> 24] + static_cast<size_t>(mt & 0xFFFFFF) * KB;
+    for (int kb = 0; kb < KB; ++kb) p.sa_t[static_cast<size_t>(kb) * p.rpad + r] = __ldg(src + kb);
   }
 }
 

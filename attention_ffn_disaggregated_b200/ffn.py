@@ -216,7 +216,8 @@ class FfnLayer:
             raise AfdError(rc, "afd_ffn_set_wait_limit")
 
     def set_tiling(self, tiling: int):
-        """0: chosen per call on the device; 1: single-CTA tiles; 2: CTA-pair tiles."""
+        """0: default (1); 1: single-CTA tiles; 2: CTA-pair tiles; 3: single-CTA tiles with the
+        W13 rows gathered from the slabs by TMA (no expert-ordered row copy)."""
         rc = lib().afd_ffn_set_tiling(self.plan, int(tiling))
         if rc != AFD_OK:
             raise AfdError(rc, "afd_ffn_set_tiling")

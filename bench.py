@@ -454,7 +454,8 @@ def main():
                        "shared_expert": inp.shape.has_shared_expert, "top_k": inp.shape.top_k,
                        "routed_rows": R, "active_experts": active,
                        "gemm_tiling": {1: "one CTA per 128x256 tile",
-                                       2: "CTA pairs on 256x256 tiles (cta_group::2)"}[tiling],
+                                       2: "CTA pairs on 256x256 tiles (cta_group::2)",
+                                       3: "one CTA per 128x256 tile, W13 rows by tile::gather4"}[tiling],
                        "l2": "flushed between steps (256 MiB write, untimed)",
                        "launch": "CUDA graph replay" if args.graph else "direct launches",
                        "parallelism": f"replica x{world}"},

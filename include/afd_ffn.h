@@ -78,8 +78,10 @@ typedef enum {
 #define AFD_MAX_GROUPS 1024 /* num_local_experts + has_shared_expert */
 #define AFD_QBLOCK 128      /* quantisation block edge */
 
-/* Timed stages of one layer call, in launch order (for afd_ffn_get_kernel_times); the
- * two GEMM stages each cover the launches of both tilings. */
+/* Timed stages of one layer call, in launch order (for afd_ffn_get_kernel_times). One
+ * kernel per stage. The gather stage copies the routed FP8 rows and their scales into
+ * expert order; with tiling 3 it moves only the scales (the W13 kernel then fetches the
+ * rows from the slabs itself). */
 #define AFD_KERNEL_ROUTE_COUNT 0
 #define AFD_KERNEL_ROUTE_SCAN 1
 #define AFD_KERNEL_ROUTE_SCATTER 2
@@ -200,10 +202,16 @@ AFD_API afd_status_t afd_ffn_set_timing(afd_ffn_plan_t plan, int32_t enable);
 AFD_API afd_status_t afd_ffn_get_kernel_times(afd_ffn_plan_t plan, float* ms);
 
 /*
- * Tiling of the two grouped GEMMs. 0 (default) or 1: one CTA per 128-row x 256-column
- * tile; 2: CTA pairs on 256-row tiles (cta_group::2 MMAs, less operand traffic per MMA,
- * but a per-K-block handshake between the two SMs that measured about 2x slower).
- * Results are the same within rounding; tiling 2 exists for tests and measurements.
+ * Tiling of the two grouped GEMMs, chosen on the host for the following calls.
+ * 0 (default) or 1: one CTA per 128-row x 256-column tile, A rows from the gather stage's
+ * expert-ordered copy.
+ * 2: CTA pairs on 256-row tiles (cta_group::2 MMAs, less operand traffic per MMA, but a
+ *    per-K-block handshake between the two SMs that measured about 2x slower).
+ * 3: as 1, but the W13 kernel fetches its A rows straight from the slabs with TMA
+ *    tile::gather4 (no row copy; 32 four-row requests per A tile, measured about 2.7x
+ *    slower for W13 on a 4096-token DeepSeek-V3 share).
+ * Results are the same within rounding; tilings 2 and 3 exist for tests and measurements.
+ * Returns AFD_ERR_INVALID_ARGUMENT outside 0..3.
  */
 AFD_API afd_status_t afd_ffn_set_tiling(afd_ffn_plan_t plan, int32_t tiling);
 
