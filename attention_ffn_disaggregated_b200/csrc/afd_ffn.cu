@@ -61,6 +61,7 @@ struct afd_ffn_plan_s {
   float *row_w, *sa_t, *sh_t, *acc;
   uint8_t *a_perm, *hq;
   int* status;
+  int* scan_ticket;   // route_count's last-block counter, zero between calls
   CUtensorMap tm_a13, tm_w13, tm_a2, tm_w2;
   // tiling 3 (W13 rows gathered from the slabs): one map per slab, re-encoded when a slab's
   // row pointer changes between calls
@@ -88,8 +89,8 @@ const char* afd_status_string(afd_status_t s) {
   return "unknown";
 }
 
-// route count, scan, scatter, gather, W13, W2, finalize
-int32_t afd_ffn_kernels_per_layer(void) { return 7; }
+// route count (+ scan), scatter, gather, W13, W2, finalize
+int32_t afd_ffn_kernels_per_layer(void) { return 6; }
 
 afd_status_t afd_ffn_check_config(const afd_ffn_config_t* c) {
   if (!c) return AFD_ERR_INVALID_ARGUMENT;
@@ -216,6 +217,7 @@ afd_status_t afd_ffn_plan(const afd_ffn_config_t* cfg, const afd_ffn_weights_t* 
   const size_t o_slab_base = take(sizeof(int32_t) * (cfg->num_slabs + 1), 16);
   const size_t o_info = take(sizeof(int32_t) * 16, 16);
   const size_t o_status = take(sizeof(int32_t) * 4, 16);
+  const size_t o_ticket = take(sizeof(int32_t) * 4, 16);
   const size_t o_chunk_hist = take(sizeof(int32_t) * P->num_chunks * El1, 16);
   const size_t o_chunk_off = take(sizeof(int32_t) * P->num_chunks * El1, 16);
   const size_t o_group_count = take(sizeof(int32_t) * (P->G + 1), 16);
@@ -249,6 +251,7 @@ afd_status_t afd_ffn_plan(const afd_ffn_config_t* cfg, const afd_ffn_weights_t* 
   P->slab_base = reinterpret_cast<int32_t*>(b + o_slab_base);
   P->info = reinterpret_cast<int32_t*>(b + o_info);
   P->status = reinterpret_cast<int*>(b + o_status);
+  P->scan_ticket = reinterpret_cast<int*>(b + o_ticket);
   P->chunk_hist = reinterpret_cast<int32_t*>(b + o_chunk_hist);
   P->chunk_off = reinterpret_cast<int32_t*>(b + o_chunk_off);
   P->group_count = reinterpret_cast<int32_t*>(b + o_group_count);
@@ -366,6 +369,7 @@ static void fill_route_params(afd_ffn_plan_t P, const int32_t* d_counts, RoutePa
   rp.group_off = P->group_off;
   rp.mtile_off = P->mtile_off;
   rp.mtile2_off = P->mtile2_off;
+  rp.scan_ticket = P->scan_ticket;
   rp.tiling = P->tiling;
   rp.tok_mt = P->tok_mt;
   rp.tok_need = P->tok_need;
@@ -460,9 +464,9 @@ afd_status_t afd_ffn_layer(afd_ffn_plan_t P, const afd_slab_t* slabs, const int3
 
   const bool tm = P->timing;
   if (tm) cudaEventRecord(P->ev[0], stream);
+  // the routing scan runs in route_count's last block (its stage time reads as zero)
   route_count_kernel<<<P->num_chunks, kRouteThreads, 0, stream>>>(rp, tab);
   if (tm) cudaEventRecord(P->ev[1], stream);
-  route_scan_kernel<<<1, 1024, 0, stream>>>(rp);
   if (tm) cudaEventRecord(P->ev[2], stream);
   route_scatter_kernel<<<P->num_chunks, kRouteThreads, P->scatter_smem, stream>>>(rp, tab);
   if (tm) cudaEventRecord(P->ev[3], stream);

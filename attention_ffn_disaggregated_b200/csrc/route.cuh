@@ -40,6 +40,7 @@ struct RouteParams {
   int32_t* group_off;     // [G+1]
   int32_t* mtile_off;     // [G+1] 128-row m-tiles
   int32_t* mtile2_off;    // [G+1] 256-row m-tiles (CTA-pair tiling); may be null
+  int* scan_ticket;       // zero between calls: route_count runs the scan; null: separate
   int tiling;             // as set on the plan: 0 (default, = 1), 1, 2 or 3
   int32_t* tok_mt;        // [Tmax] (slab << 24) | row
   int32_t* tok_need;      // [Tmax] contributions this GPU adds to the token
@@ -103,41 +104,7 @@ __device__ __forceinline__ uint32_t classify_token(const int32_t* ids, int K, in
   return mask;
 }
 
-// 1. per-chunk histogram of local groups; token bookkeeping.
-__global__ void __launch_bounds__(kRouteThreads) route_count_kernel(
-    const __grid_constant__ RouteParams p, const __grid_constant__ SlabTable slabs) {
-  __shared__ int32_t s_base[AFD_MAX_SLABS + 1];
-  __shared__ int32_t s_hist[AFD_MAX_GROUPS];
-  load_slab_base(p, s_base);
-  const int T = s_base[p.M];
-  if (blockIdx.x == 0) {
-    for (int m = threadIdx.x; m <= p.M; m += blockDim.x) p.slab_base[m] = s_base[m];
-    if (threadIdx.x == 0) p.info[0] = T;
-  }
-  for (int e = threadIdx.x; e < p.El; e += blockDim.x) s_hist[e] = 0;
-  __syncthreads();
-  const int g = blockIdx.x * kChunkTokens + threadIdx.x;
-  if (g < T) {
-    const int m = find_slab(s_base, p.M, g);
-    const int t = g - s_base[m];
-    int32_t ids[AFD_MAX_TOP_K];
-    int le[AFD_MAX_TOP_K];
-    const int32_t* src = slabs.ids[m] + static_cast<size_t>(t) * p.K;
-    for (int k = 0; k < p.K; ++k) ids[k] = src[k];
-    bool bad = false;
-    uint32_t mask = classify_token(ids, p.K, p.e0, p.El, p.Eg, le, &bad);
-    for (int k = 0; k < p.K; ++k)
-      if (mask >> k & 1u) atomicAdd(&s_hist[le[k]], 1);
-    p.tok_mt[g] = (m << 24) | t;
-    p.tok_need[g] = __popc(mask) + p.S;
-    if (bad) atomicOr(p.status, AFD_STATUS_BAD_ROUTING);
-  }
-  __syncthreads();
-  int32_t* out = p.chunk_hist + static_cast<size_t>(blockIdx.x) * max(p.El, 1);
-  for (int e = threadIdx.x; e < p.El; e += blockDim.x) out[e] = s_hist[e];
-}
-
-// Block-wide exclusive scan of one value per thread (blockDim.x == 1024).
+// Block-wide exclusive scan of one value per thread (whole warps, up to 1024 threads).
 __device__ __forceinline__ int block_exclusive_scan(int v, int* s_warp, int* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int x = v;
@@ -164,10 +131,9 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* s_warp, int* tot
   return excl;
 }
 
-// 2. chunk offsets per group, group offsets (exclusive scan) and the m-tile schedule.
-__global__ void __launch_bounds__(1024) route_scan_kernel(const __grid_constant__ RouteParams p) {
-  __shared__ int s_warp[32];
-  const int T = p.info[0];
+// 2. chunk offsets per group, group offsets (exclusive scan) and the m-tile schedule,
+// computed by one block of any whole-warp size.
+__device__ void route_scan_body(const RouteParams& p, int T, int* s_warp) {
   const int chunks = (T + kChunkTokens - 1) / kChunkTokens;
   const int El1 = max(p.El, 1);
   for (int e = threadIdx.x; e < p.El; e += blockDim.x) {
@@ -210,6 +176,59 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(const __grid_constant_
     // the tiling this call runs (the host launches only its kernels)
     p.info[3] = p.tiling == 0 ? 1 : p.tiling;
   }
+}
+
+// 2 as its own launch (one block of 1024 threads).
+__global__ void __launch_bounds__(1024) route_scan_kernel(const __grid_constant__ RouteParams p) {
+  __shared__ int s_warp[32];
+  route_scan_body(p, p.info[0], s_warp);
+}
+
+// 1. per-chunk histogram of local groups; token bookkeeping. With p.scan_ticket set, the
+// block that finishes last also runs step 2 (every block publishes its histogram, fences,
+// then takes a ticket; the counter is returned to zero for the next call).
+__global__ void __launch_bounds__(kRouteThreads) route_count_kernel(
+    const __grid_constant__ RouteParams p, const __grid_constant__ SlabTable slabs) {
+  __shared__ int32_t s_base[AFD_MAX_SLABS + 1];
+  __shared__ int32_t s_hist[AFD_MAX_GROUPS];
+  load_slab_base(p, s_base);
+  const int T = s_base[p.M];
+  if (blockIdx.x == 0) {
+    for (int m = threadIdx.x; m <= p.M; m += blockDim.x) p.slab_base[m] = s_base[m];
+    if (threadIdx.x == 0) p.info[0] = T;
+  }
+  for (int e = threadIdx.x; e < p.El; e += blockDim.x) s_hist[e] = 0;
+  __syncthreads();
+  const int g = blockIdx.x * kChunkTokens + threadIdx.x;
+  if (g < T) {
+    const int m = find_slab(s_base, p.M, g);
+    const int t = g - s_base[m];
+    int32_t ids[AFD_MAX_TOP_K];
+    int le[AFD_MAX_TOP_K];
+    const int32_t* src = slabs.ids[m] + static_cast<size_t>(t) * p.K;
+    for (int k = 0; k < p.K; ++k) ids[k] = src[k];
+    bool bad = false;
+    uint32_t mask = classify_token(ids, p.K, p.e0, p.El, p.Eg, le, &bad);
+    for (int k = 0; k < p.K; ++k)
+      if (mask >> k & 1u) atomicAdd(&s_hist[le[k]], 1);
+    p.tok_mt[g] = (m << 24) | t;
+    p.tok_need[g] = __popc(mask) + p.S;
+    if (bad) atomicOr(p.status, AFD_STATUS_BAD_ROUTING);
+  }
+  __syncthreads();
+  int32_t* out = p.chunk_hist + static_cast<size_t>(blockIdx.x) * max(p.El, 1);
+  for (int e = threadIdx.x; e < p.El; e += blockDim.x) out[e] = s_hist[e];
+  if (!p.scan_ticket) return;
+  __shared__ int s_last;
+  __shared__ int s_warp[32];
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) s_last = atomicAdd(p.scan_ticket, 1) == static_cast<int>(gridDim.x) - 1;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  route_scan_body(p, T, s_warp);
+  if (threadIdx.x == 0) *p.scan_ticket = 0;
 }
 
 // 3. stable placement of every local (token, slot) pair and of the shared rows.
@@ -306,33 +325,68 @@ __global__ void __launch_bounds__(kRouteThreads) route_scatter_kernel(
 }
 
 // 4. copy routed rows (FP8 codes and their per-128 scales) into expert order.
-// One warp per row; scales are stored transposed ([H/128][rpad]) so that a GEMM tile
-// reads one block's scales for 32 consecutive rows with one coalesced load.
+// One warp per token: the token's row is read once, 4 KiB at a time (eight 16-byte loads
+// in flight per lane), and written to each of its destination rows (its local top-K
+// slots, then its shared-expert row). Scales are stored transposed ([H/128][rpad]) so
+// that a GEMM tile reads one block's scales for 32 consecutive rows with one load.
 __global__ void __launch_bounds__(kRouteThreads) gather_rows_kernel(
     const __grid_constant__ RouteParams p, const __grid_constant__ SlabTable slabs) {
-  const int R = p.info[1];
+  const int T = p.info[0];
+  const int K = p.K;
   const int lane = threadIdx.x & 31;
   const int nwarps = (gridDim.x * blockDim.x) >> 5;
   const int KB = p.H / AFD_QBLOCK;
-  for (int r = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; r < R; r += nwarps) {
-    const int g = p.row_token[r];
+  const int n16 = p.H / 16;               // H is a multiple of 256: n16 a multiple of 16
+  for (int g = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; g < T; g += nwarps) {
     const int mt = p.tok_mt[g];
     const int m = mt >> 24, t = mt & 0xFFFFFF;
+    // destination rows: lane k < K holds slot k's row (or -1), the shared row follows
+    int myrow = -1;
+    if (lane < K) myrow = p.pos[static_cast<size_t>(g) * K + lane];
+    unsigned dmask = __ballot_sync(0xffffffffu, myrow >= 0);
+    const int shared_row = p.S ? p.group_off[p.El] + g : -1;
     const uint4* __restrict__ src =
         reinterpret_cast<const uint4*>(slabs.x[m] + static_cast<size_t>(t) * p.H);
-    uint4* __restrict__ dst = reinterpret_cast<uint4*>(p.a_perm + static_cast<size_t>(r) * p.H);
-    const int n16 = p.H / 16;             // H is a multiple of 256: n16 a multiple of 16
-    int i = lane;
-    for (; i + 7 * 32 < n16; i += 8 * 32) {   // eight 16-byte loads in flight per lane
+    for (int i0 = 0; i0 < n16; i0 += 8 * 32) {
       uint4 v[8];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) v[j] = __ldg(src + i + 32 * j);
+      for (int j = 0; j < 8; ++j) {
+        const int i = i0 + 32 * j + lane;
+        if (i < n16) v[j] = __ldg(src + i);
+      }
+      unsigned d = dmask;
+      int r = -1;
+      while (true) {
+        if (d) {
+          const int k = __ffs(d) - 1;
+          d &= d - 1;
+          r = __shfl_sync(0xffffffffu, myrow, k);
+        } else if (r != shared_row) {
+          r = shared_row;
+        } else {
+          break;
+        }
+        if (r < 0) break;
+        uint4* __restrict__ dst = reinterpret_cast<uint4*>(p.a_perm + static_cast<size_t>(r) * p.H);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) dst[i + 32 * j] = v[j];
+        for (int j = 0; j < 8; ++j) {
+          const int i = i0 + 32 * j + lane;
+          if (i < n16) dst[i] = v[j];
+        }
+      }
     }
-    for (; i < n16; i += 32) dst[i] = __ldg(src + i);
     const float* ssrc = slabs.xs[m] + static_cast<size_t>(t) * KB;
-    for (int kb = lane; kb < KB; kb += 32) p.sa_t[static_cast<size_t>(kb) * p.rpad + r] = ssrc[kb];
+    for (int kb = lane; kb < KB; kb += 32) {
+      const float sc = ssrc[kb];
+      float* dcol = p.sa_t + static_cast<size_t>(kb) * p.rpad;
+      unsigned d = dmask;
+      while (d) {
+        const int k = __ffs(d) - 1;
+        d &= d - 1;
+        dcol[p.pos[static_cast<size_t>(g) * K + k]] = sc;
+      }
+      if (shared_row >= 0) dcol[shared_row] = sc;
+    }
   }
 }
 

@@ -79,9 +79,11 @@ typedef enum {
 #define AFD_QBLOCK 128      /* quantisation block edge */
 
 /* Timed stages of one layer call, in launch order (for afd_ffn_get_kernel_times). One
- * kernel per stage. The gather stage copies the routed FP8 rows and their scales into
- * expert order; with tiling 3 it moves only the scales (the W13 kernel then fetches the
- * rows from the slabs itself). */
+ * kernel per stage, except that the routing scan runs in the last block of the route
+ * count kernel: AFD_KERNEL_ROUTE_COUNT covers both and AFD_KERNEL_ROUTE_SCAN reads as
+ * zero. The gather stage copies the routed FP8 rows and their scales into expert order;
+ * with tiling 3 it moves only the scales (the W13 kernel then fetches the rows from the
+ * slabs itself). */
 #define AFD_KERNEL_ROUTE_COUNT 0
 #define AFD_KERNEL_ROUTE_SCAN 1
 #define AFD_KERNEL_ROUTE_SCATTER 2
