@@ -62,6 +62,7 @@ struct afd_ffn_plan_s {
   uint8_t *a_perm, *hq;
   int* status;
   int* scan_ticket;   // route_count's last-block counter, zero between calls
+  int32_t* ready;     // fused W13->W2 launch: per m-tile readiness counters
   CUtensorMap tm_a13, tm_w13, tm_a2, tm_w2;
   // tiling 3 (W13 rows gathered from the slabs): one map per slab, re-encoded when a slab's
   // row pointer changes between calls
@@ -89,7 +90,7 @@ const char* afd_status_string(afd_status_t s) {
   return "unknown";
 }
 
-// route count (+ scan), scatter, gather, W13, W2, finalize
+// default tiling: route count (+ scan), scatter, gather, W13, W2, finalize
 int32_t afd_ffn_kernels_per_layer(void) { return 6; }
 
 afd_status_t afd_ffn_check_config(const afd_ffn_config_t* c) {
@@ -178,7 +179,8 @@ afd_status_t afd_ffn_plan(const afd_ffn_config_t* cfg, const afd_ffn_weights_t* 
   // The GEMM kernels split the block's registers between warpgroups with setmaxnreg; that
   // is only safe when the block is launched with exactly the budget the split assumes.
   {
-    const void* fns[5] = {reinterpret_cast<const void*>(grouped_gemm_kernel<EPI_SWIGLU, 1, false>),
+    const void* fns[6] = {reinterpret_cast<const void*>(grouped_gemm_kernel<EPI_FUSED, 1, false>),
+                          reinterpret_cast<const void*>(grouped_gemm_kernel<EPI_SWIGLU, 1, false>),
                           reinterpret_cast<const void*>(grouped_gemm_kernel<EPI_SWIGLU, 1, true>),
                           reinterpret_cast<const void*>(grouped_gemm_kernel<EPI_SWIGLU, 2, false>),
                           reinterpret_cast<const void*>(grouped_gemm_kernel<EPI_COMBINE, 1, false>),
@@ -218,6 +220,7 @@ afd_status_t afd_ffn_plan(const afd_ffn_config_t* cfg, const afd_ffn_weights_t* 
   const size_t o_info = take(sizeof(int32_t) * 16, 16);
   const size_t o_status = take(sizeof(int32_t) * 4, 16);
   const size_t o_ticket = take(sizeof(int32_t) * 4, 16);
+  const size_t o_ready = take(sizeof(int32_t) * (P->rpad / 128 + P->G + 1), 16);
   const size_t o_chunk_hist = take(sizeof(int32_t) * P->num_chunks * El1, 16);
   const size_t o_chunk_off = take(sizeof(int32_t) * P->num_chunks * El1, 16);
   const size_t o_group_count = take(sizeof(int32_t) * (P->G + 1), 16);
@@ -252,6 +255,7 @@ afd_status_t afd_ffn_plan(const afd_ffn_config_t* cfg, const afd_ffn_weights_t* 
   P->info = reinterpret_cast<int32_t*>(b + o_info);
   P->status = reinterpret_cast<int*>(b + o_status);
   P->scan_ticket = reinterpret_cast<int*>(b + o_ticket);
+  P->ready = reinterpret_cast<int32_t*>(b + o_ready);
   P->chunk_hist = reinterpret_cast<int32_t*>(b + o_chunk_hist);
   P->chunk_off = reinterpret_cast<int32_t*>(b + o_chunk_off);
   P->group_count = reinterpret_cast<int32_t*>(b + o_group_count);
@@ -282,7 +286,9 @@ afd_status_t afd_ffn_plan(const afd_ffn_config_t* cfg, const afd_ffn_weights_t* 
     return st;
   }
   P->scatter_smem = sizeof(int32_t) * (static_cast<size_t>(kRouteWarps) * El1 + kRouteWarps * 32 * K);
-  if (cudaFuncSetAttribute(grouped_gemm_kernel<EPI_SWIGLU, 1, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (cudaFuncSetAttribute(grouped_gemm_kernel<EPI_FUSED, 1, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(gemm_smem_bytes(EPI_FUSED))) != cudaSuccess ||
+      cudaFuncSetAttribute(grouped_gemm_kernel<EPI_SWIGLU, 1, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(gemm_smem_bytes(EPI_SWIGLU))) != cudaSuccess ||
       cudaFuncSetAttribute(grouped_gemm_kernel<EPI_SWIGLU, 1, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(gemm_smem_bytes(EPI_SWIGLU))) != cudaSuccess ||
@@ -370,6 +376,7 @@ static void fill_route_params(afd_ffn_plan_t P, const int32_t* d_counts, RoutePa
   rp.mtile_off = P->mtile_off;
   rp.mtile2_off = P->mtile2_off;
   rp.scan_ticket = P->scan_ticket;
+  rp.ready = P->ready;
   rp.tiling = P->tiling;
   rp.tok_mt = P->tok_mt;
   rp.tok_need = P->tok_need;
@@ -439,10 +446,11 @@ afd_status_t afd_ffn_layer(afd_ffn_plan_t P, const afd_slab_t* slabs, const int3
     tab.y[m] = static_cast<__nv_bfloat16*>(s.y);
     ytab.y[m] = static_cast<__nv_bfloat16*>(s.y);
   }
-  // tilings 1 (default) and 2 read an expert-ordered copy of the rows made by the gather
-  // stage; tiling 3 gathers them from the slabs inside the W13 kernel (tile::gather4)
+  // tilings 1 (default), 2 and 4 (W13 and W2 in one persistent launch) read an
+  // expert-ordered copy of the rows made by the gather stage; tiling 3 gathers them from
+  // the slabs inside the W13 kernel (tile::gather4)
   const int tiling = P->tiling == 0 ? 1 : P->tiling;
-  const bool pair = tiling == 2, slab_gather = tiling == 3;
+  const bool pair = tiling == 2, slab_gather = tiling == 3, fused = tiling == 4;
   if (slab_gather) {
     EncodeTiledFn enc = get_encode_fn();
     if (!enc) return AFD_ERR_CUDA;
@@ -474,7 +482,17 @@ afd_status_t afd_ffn_layer(afd_ffn_plan_t P, const afd_slab_t* slabs, const int3
   else gather_rows_kernel<<<P->num_sms * 8, kRouteThreads, 0, stream>>>(rp, tab);
   if (tm) cudaEventRecord(P->ev[4], stream);
   const int grid1 = P->num_sms, grid2 = P->num_sms & ~1;
-  if (slab_gather) {
+  if (fused) {
+    // one persistent launch: every W13 tile, then every W2 tile (the W2 stage time reads
+    // as zero)
+    FusedArgs fa;
+    fa.p2 = g2;
+    fa.tm_a2 = P->tm_a2;
+    fa.tm_b2 = P->tm_w2;
+    fa.ready = P->ready;
+    grouped_gemm_kernel<EPI_FUSED, 1, false><<<grid1, kGemmThreads, gemm_smem_bytes(EPI_FUSED), stream>>>(
+        g13, P->tm_a13, P->tm_w13, ytab, fa);
+  } else if (slab_gather) {
     grouped_gemm_kernel<EPI_SWIGLU, 1, true><<<grid1, kGemmThreads, gemm_smem_bytes(EPI_SWIGLU), stream>>>(
         g13, P->tm_a13, P->tm_w13, ytab, P->slab_maps);
   } else if (!pair) {
@@ -485,11 +503,12 @@ afd_status_t afd_ffn_layer(afd_ffn_plan_t P, const afd_slab_t* slabs, const int3
     return AFD_ERR_CUDA;
   }
   if (tm) cudaEventRecord(P->ev[5], stream);
-  if (!pair) {
+  if (!fused && !pair) {
     grouped_gemm_kernel<EPI_COMBINE, 1, false><<<grid1, kGemmThreads, gemm_smem_bytes(EPI_COMBINE), stream>>>(
         g2, P->tm_a2, P->tm_w2, ytab, AMaps<false>{0});
-  } else if (launch_pair(grouped_gemm_kernel<EPI_COMBINE, 2, false>, grid2, gemm_smem_bytes(EPI_COMBINE),
-                         stream, g2, P->tm_a2, P->tm_w2, ytab) != cudaSuccess) {
+  } else if (pair && launch_pair(grouped_gemm_kernel<EPI_COMBINE, 2, false>, grid2,
+                                 gemm_smem_bytes(EPI_COMBINE), stream, g2, P->tm_a2, P->tm_w2,
+                                 ytab) != cudaSuccess) {
     return AFD_ERR_CUDA;
   }
   if (tm) cudaEventRecord(P->ev[6], stream);
@@ -584,7 +603,7 @@ afd_status_t afd_ffn_set_wait_limit(afd_ffn_plan_t P, int64_t limit_ns) {
 }
 
 afd_status_t afd_ffn_set_tiling(afd_ffn_plan_t P, int32_t tiling) {
-  if (!P || tiling < 0 || tiling > 3) return AFD_ERR_INVALID_ARGUMENT;
+  if (!P || tiling < 0 || tiling > 4) return AFD_ERR_INVALID_ARGUMENT;
   P->tiling = tiling;
   return AFD_OK;
 }

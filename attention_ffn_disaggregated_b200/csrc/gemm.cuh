@@ -54,7 +54,9 @@ constexpr int kEpilogueRegs = 232;
 static_assert(128 * kProducerRegs + 256 * kEpilogueRegs <= kGemmThreads * kLaunchRegs,
               "register split exceeds the launch allocation");
 
-enum EpiKind { EPI_SWIGLU = 0, EPI_COMBINE = 1 };
+// EPI_FUSED: one launch runs every W13 tile (SWIGLU epilogue) and then every W2 tile
+// (COMBINE epilogue), single-CTA tiles; see FusedArgs.
+enum EpiKind { EPI_SWIGLU = 0, EPI_COMBINE = 1, EPI_FUSED = 2 };
 
 template <int PAIR>
 struct Tiling {
@@ -79,11 +81,7 @@ template <>
 struct AMaps<false> {
   int unused;
 };
-template <bool GATHER>
-__device__ __forceinline__ const CUtensorMap* slab_map(const AMaps<GATHER>& a, int m) {
-  if constexpr (GATHER) return &a.m[m];
-  else return nullptr;
-}
+
 
 struct GemmParams {
   const int32_t* info;        // [0] tokens, [1] rows, [2] m-tiles of this call
@@ -113,6 +111,58 @@ struct GemmParams {
   int inject_stall;
 };
 
+// The fused launch's second projection. W2 tile (mt, nt) reads the h rows of m-tile mt,
+// written by the epilogues of the W13 tiles (mt, 0 .. p.n_tiles-1): each of their 8
+// epilogue warps adds 1 to ready[mt] (release) after its stores, and the W2 tile's
+// producer and epilogue wait (bounded, acquire) for 8 * p.n_tiles. Every CTA walks its
+// tiles in increasing order and all W13 tiles precede all W2 tiles, so a W13 tile never
+// waits for anything and every wait ends.
+struct FusedArgs {
+  GemmParams p2;
+  CUtensorMap tm_a2;          // h codes [rpad][I]
+  CUtensorMap tm_b2;          // W2 codes [E][H][I]
+  int32_t* ready;             // [m-tiles], zeroed by the routing scan of each call
+};
+
+template <int EPI, bool GATHER>
+struct ExtraArg {
+  using type = AMaps<GATHER>;
+};
+template <>
+struct ExtraArg<EPI_FUSED, false> {
+  using type = FusedArgs;
+};
+
+__device__ __forceinline__ const CUtensorMap* slab_map(const AMaps<true>& a, int m) { return &a.m[m]; }
+__device__ __forceinline__ const CUtensorMap* slab_map(const AMaps<false>&, int) { return nullptr; }
+__device__ __forceinline__ const CUtensorMap* slab_map(const FusedArgs&, int) { return nullptr; }
+
+// Parameters and operand maps of a tile: the launch's own, or (fused, W2 tile) the
+// second projection's.
+template <class X>
+__device__ __forceinline__ const GemmParams& tile_params(bool w2, const GemmParams& p, const X&) {
+  return p;
+}
+__device__ __forceinline__ const GemmParams& tile_params(bool w2, const GemmParams& p,
+                                                         const FusedArgs& x) {
+  return w2 ? x.p2 : p;
+}
+template <class X>
+__device__ __forceinline__ void tile_maps(bool, const CUtensorMap* a, const CUtensorMap* b, const X&,
+                                          const CUtensorMap** ma, const CUtensorMap** mb) {
+  *ma = a;
+  *mb = b;
+}
+__device__ __forceinline__ void tile_maps(bool w2, const CUtensorMap* a, const CUtensorMap* b,
+                                          const FusedArgs& x, const CUtensorMap** ma,
+                                          const CUtensorMap** mb) {
+  *ma = w2 ? &x.tm_a2 : a;
+  *mb = w2 ? &x.tm_b2 : b;
+}
+template <class X>
+__device__ __forceinline__ int* ready_of(const X&) { return nullptr; }
+__device__ __forceinline__ int* ready_of(const FusedArgs& x) { return x.ready; }
+
 // 16-byte multiple: the combine staging that follows it is accessed as float4
 struct alignas(16) GemmSmem {
   uint64_t full[kMaxStages];
@@ -133,7 +183,7 @@ static_assert(Tiling<2>::kStages * Tiling<2>::kStageBytes == kGemmSmemTiles, "ti
 constexpr size_t kStgBytes = static_cast<size_t>(kEpiWarps) * 16 * kStgStride * sizeof(float);
 
 __host__ __device__ constexpr size_t gemm_smem_bytes(int epi) {
-  return 1024 + kGemmSmemTiles + sizeof(GemmSmem) + (epi == EPI_COMBINE ? kStgBytes : 0);
+  return 1024 + kGemmSmemTiles + sizeof(GemmSmem) + (epi != EPI_SWIGLU ? kStgBytes : 0);
 }
 
 // A wait that ignores the abort flag; used only to drain copies/MMAs already in flight.
@@ -146,7 +196,7 @@ __device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity, 
 }
 
 struct TileCoord {
-  int e, row0, rows, nt;
+  int e, row0, rows, nt, mt;
 };
 
 // Tile -> (expert, first row of this CTA's 128 rows, valid rows, column tile).
@@ -156,6 +206,7 @@ __device__ __forceinline__ TileCoord decode_tile(int tile, int n_tiles, const in
                                                  int G, const int32_t* group_off, int rank) {
   TileCoord c;
   const int mt = tile / n_tiles;
+  c.mt = mt;
   c.nt = tile - mt * n_tiles;
   int lo = 0, hi = G - 1;               // last group whose first m-tile is <= mt
   while (lo < hi) {
@@ -170,15 +221,18 @@ __device__ __forceinline__ TileCoord decode_tile(int tile, int n_tiles, const in
 }
 
 // GATHER (W13, single-CTA tiles only): the A tile's rows are fetched from the slabs
-// through `amaps` instead of from the expert-ordered copy behind `tm_a`.
+// through `extra` (AMaps<true>) instead of from the expert-ordered copy behind `tm_a`.
+// EPI_FUSED: `p`, `tm_a`, `tm_b` describe W13 and `extra` (FusedArgs) W2.
 template <int EPI, int PAIR, bool GATHER>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ GemmParams p,
                         const __grid_constant__ CUtensorMap tm_a,
                         const __grid_constant__ CUtensorMap tm_b,
                         const __grid_constant__ YTable ytab,
-                        const __grid_constant__ AMaps<GATHER> amaps) {
+                        const __grid_constant__ typename ExtraArg<EPI, GATHER>::type extra) {
   static_assert(!GATHER || (EPI == EPI_SWIGLU && PAIR == 1), "slab gather: W13, single-CTA tiles");
+  static_assert(EPI != EPI_FUSED || (PAIR == 1 && !GATHER), "fused launch: single-CTA tiles");
+  constexpr bool kFused = EPI == EPI_FUSED;
   using TL = Tiling<PAIR>;
   constexpr int kStages = TL::kStages;
 
@@ -227,7 +281,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (PAIR == 2) cluster_sync();     // both CTAs' barriers exist before any remote signal
   tc_fence_after();
   const uint32_t tmem_base = S.tmem_base;
-  const int total_tiles = S.mtile[p.G] * p.n_tiles;
+  // tile sequence: the launch's own tiles [0, T1) and, fused, the W2 tiles after them
+  const int T1 = S.mtile[p.G] * p.n_tiles;
+  int total_tiles = T1;
+  if constexpr (kFused) total_tiles += S.mtile[p.G] * extra.p2.n_tiles;
+  int* ready = ready_of(extra);
+  const int ready_target = kEpiWarps * p.n_tiles;
 
   if (warp < 4) {
     // each role's code sits inside the branch that sets its register budget
@@ -278,12 +337,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
           __syncwarp();
           if (one_slab) {
-            tma_gather4(a, slab_map(amaps, rm[0]), &S.full[s], kb * kBK, rt[0], rt[1], rt[2], rt[3],
+            tma_gather4(a, slab_map(extra, rm[0]), &S.full[s], kb * kBK, rt[0], rt[1], rt[2], rt[3],
                         pol_a);
           } else {
 #pragma unroll
             for (int j = 0; j < 4; ++j)
-              tma_load_2d(a + j * kBK, slab_map(amaps, rm[j]), &S.full[s], kb * kBK, rt[j], pol_a);
+              tma_load_2d(a + j * kBK, slab_map(extra, rm[j]), &S.full[s], kb * kBK, rt[j], pol_a);
           }
         }
       }
@@ -301,22 +360,39 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       // A rows are re-read by every column tile of their m-tile; in the down projection
       // the weights stream past the L2-resident combine accumulators, so they go first
       const uint64_t pol_a = policy_evict_last();
-      const uint64_t pol_b = EPI == EPI_COMBINE ? policy_evict_first() : policy_evict_last();
       int it = 0;
       bool ok = true;
       int skipped = -1;
       for (int tile = unit; ok && tile < total_tiles; tile += nunits) {
-        const TileCoord c = decode_tile<PAIR>(tile, p.n_tiles, S.mtile, p.G, p.group_off, rank);
+        const bool w2 = kFused && tile >= T1;
+        const GemmParams& tp = tile_params(w2, p, extra);
+        const CUtensorMap *ma, *mb;
+        tile_maps(w2, &tm_a, &tm_b, extra, &ma, &mb);
+        const TileCoord c = decode_tile<PAIR>(w2 ? tile - T1 : tile, tp.n_tiles, S.mtile, p.G,
+                                              p.group_off, rank);
+        const bool swiglu = EPI == EPI_SWIGLU || (kFused && !w2);
         // B rows of this tile: [brow0, +128) and [brow1, +128); a pair splits them
         int brow0, brow1;
-        if (EPI == EPI_SWIGLU) {
+        if (swiglu) {
           brow0 = c.nt * 128;               // gate block
-          brow1 = p.I + c.nt * 128;         // up block
+          brow1 = tp.I + c.nt * 128;         // up block
         } else {
           brow0 = c.nt * kBN;
           brow1 = c.nt * kBN + 128;
         }
-        for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
+        const uint64_t pol_b = swiglu ? policy_evict_last() : policy_evict_first();
+        // loop bounds in registers: the asm memory clobbers of the waits below would
+        // otherwise force reloads through the (run-time selected) parameter reference
+        const int nkb = kFused ? tp.num_kb : p.num_kb;
+        if (w2) {
+          // the h rows of this m-tile are complete once all its W13 tiles have stored them
+          if (!wait_count(ready + c.mt, ready_target, abort_flag, p.status, p.wait_limit_ns)) {
+            ok = false;
+            break;
+          }
+          fence_proxy_async_global();
+        }
+        for (int kb = 0; kb < (kFused ? nkb : p.num_kb); ++kb, ++it) {
           const int s = it % kStages;
           const uint32_t ph = (it / kStages) & 1;
           if (!mbar_wait(&S.empty[s], ph ^ 1, abort_flag, p.status, p.wait_limit_ns)) {
@@ -331,9 +407,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           uint8_t* b = sB + s * TL::kBBytes;
           if (PAIR == 1) {
             mbar_arrive_expect_tx(&S.full[s], TL::kTxBytes);
-            tma_load_2d(a, &tm_a, &S.full[s], kb * kBK, c.row0, pol_a);
-            tma_load_3d(b, &tm_b, &S.full[s], kb * kBK, brow0, c.e, pol_b);
-            tma_load_3d(b + TL::kBBytes / 2, &tm_b, &S.full[s], kb * kBK, brow1, c.e, pol_b);
+            tma_load_2d(a, ma, &S.full[s], kb * kBK, c.row0, pol_a);
+            tma_load_3d(b, mb, &S.full[s], kb * kBK, brow0, c.e, pol_b);
+            tma_load_3d(b + TL::kBBytes / 2, mb, &S.full[s], kb * kBK, brow1, c.e, pol_b);
           } else {
             const uint32_t fb = mapa_shared(smem_u32(&S.full[s]), 0);
             if (leader) mbar_arrive_expect_tx(&S.full[s], TL::kTxBytes);
@@ -355,7 +431,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int it = 0, kbg = 0;
       bool ok = true;
       for (int tile = unit; ok && tile < total_tiles; tile += nunits) {
-        for (int kb = 0; kb < p.num_kb; ++kb, ++it, ++kbg) {
+        const int num_kb = tile_params(kFused && tile >= T1, p, extra).num_kb;
+        for (int kb = 0; kb < num_kb; ++kb, ++it, ++kbg) {
           const int s = it % kStages;
           const uint32_t ph = (it / kStages) & 1;
           if (!mbar_wait(&S.full[s], ph, abort_flag, p.status, p.wait_limit_ns)) {
@@ -416,14 +493,30 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     bool ok = true;
     const uint64_t pol_acc = policy_evict_last();
     for (int tile = unit; ok && tile < total_tiles; tile += nunits, ++titer) {
-      const TileCoord c = decode_tile<PAIR>(tile, p.n_tiles, S.mtile, p.G, p.group_off, rank);
+      const bool w2 = kFused && tile >= T1;
+      const GemmParams& tp = tile_params(w2, p, extra);
+      const TileCoord c = decode_tile<PAIR>(w2 ? tile - T1 : tile, tp.n_tiles, S.mtile, p.G,
+                                            p.group_off, rank);
+      const bool swiglu = EPI == EPI_SWIGLU || (kFused && !w2);
       const int grow = c.row0 + trow;
       const bool valid = trow < c.rows;
-      const float* wsb = p.w_scale + static_cast<size_t>(c.e) * p.ws_rows * p.num_kb;
+      if (w2) {
+        // the h scales of this m-tile come from other CTAs' W13 epilogues
+        int got = 1;
+        if (lane == 0) got = wait_count(ready + c.mt, ready_target, abort_flag, p.status, p.wait_limit_ns);
+        got = __shfl_sync(0xffffffffu, got, 0);
+        if (!got) {
+          ok = false;
+          break;
+        }
+        ld_acquire(ready + c.mt);
+      }
+      const int nkb = kFused ? tp.num_kb : p.num_kb;
+      const float* wsb = tp.w_scale + static_cast<size_t>(c.e) * tp.ws_rows * nkb;
       int rs0, rs1, c0, c1;
-      if (EPI == EPI_SWIGLU) {
+      if (swiglu) {
         rs0 = c.nt;
-        rs1 = p.I / 128 + c.nt;
+        rs1 = tp.I / 128 + c.nt;
         c0 = 64 * half;
         c1 = 128 + 64 * half;
       } else {
@@ -431,21 +524,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         c0 = 128 * half;
         c1 = 128 * half + 64;
       }
-      const float* ws0 = wsb + static_cast<size_t>(rs0) * p.num_kb;
-      const float* ws1 = wsb + static_cast<size_t>(rs1) * p.num_kb;
+      const float* ws0 = wsb + static_cast<size_t>(rs0) * nkb;
+      const float* ws1 = wsb + static_cast<size_t>(rs1) * nkb;
       // acc[j] holds columns (2j, 2j+1) of this thread's 128: [0,32) from the first
       // 64-column group, [32,64) from the second
       float2 acc[64];
 #pragma unroll
       for (int i = 0; i < 64; ++i) acc[i] = make_float2(0.f, 0.f);
       // scales for K block kb+1 are fetched while block kb is processed
-      const float* sap = p.sa_t + grow;
+      const float* sap = tp.sa_t + grow;
       float sa_n = sap[0];
       float w0_n = __ldg(ws0), w1_n = __ldg(ws1);
-      for (int kb = 0; kb < p.num_kb; ++kb, ++kbg) {
+      for (int kb = 0; kb < (kFused ? nkb : p.num_kb); ++kb, ++kbg) {
         const float s0 = sa_n * w0_n;
         const float s1 = sa_n * w1_n;
-        if (kb + 1 < p.num_kb) {
+        if (kb + 1 < (kFused ? nkb : p.num_kb)) {
           sa_n = sap[static_cast<size_t>(kb + 1) * p.rpad];
           w0_n = __ldg(ws0 + kb + 1);
           w1_n = __ldg(ws1 + kb + 1);
@@ -494,7 +587,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       if (!ok) break;
 
-      if (EPI == EPI_SWIGLU) {
+      if (swiglu) {
         // h = silu(g) * u on this thread's 64 channels; block amax shared with the partner
         // warp that holds the other 64 channels of the same rows
         float amax = 0.f;
@@ -532,6 +625,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           for (int j = 0; j < 4; ++j) dst[j] = out[j];
           if (half == 0) p.sh_t[static_cast<size_t>(c.nt) * p.rpad + grow] = sc;
         }
+        if (kFused) {
+          // this warp's h rows and scales are stored: make them visible to the TMA loads
+          // and the epilogues of the W2 tiles of this m-tile
+          fence_proxy_async_global();
+          __syncwarp();
+          if (lane == 0) red_release_add(ready + c.mt, 1);
+        }
       } else {
         // weighted combine: fp32 reductions into the token accumulator (kept in L2 with
         // an evict-last hint), staged through shared memory so that each reduction covers
@@ -539,8 +639,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         int g = -1;
         float wgt = 0.f;
         if (valid) {
-          g = p.row_token[grow];
-          wgt = p.row_w[grow];
+          g = tp.row_token[grow];
+          wgt = tp.row_w[grow];
         }
         // the 32 rows go through the staging in two halves of 16; a reduction instruction
         // then covers 4 rows x 128 contiguous bytes (8 lanes per row)
@@ -566,7 +666,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               const int gg = __shfl_sync(0xffffffffu, g, 16 * hr + rl);
               const float4 v = *reinterpret_cast<const float4*>(sw + rl * kStgStride + cc);
               if (gg >= 0)
-                red_add_v4_hint(p.acc + static_cast<size_t>(gg) * p.H + col0 + 32 * ch + cc, v.x,
+                red_add_v4_hint(tp.acc + static_cast<size_t>(gg) * tp.H + col0 + 32 * ch + cc, v.x,
                                 v.y, v.z, v.w, pol_acc);
             }
             __syncwarp();

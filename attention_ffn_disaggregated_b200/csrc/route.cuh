@@ -41,6 +41,7 @@ struct RouteParams {
   int32_t* mtile_off;     // [G+1] 128-row m-tiles
   int32_t* mtile2_off;    // [G+1] 256-row m-tiles (CTA-pair tiling); may be null
   int* scan_ticket;       // zero between calls: route_count runs the scan; null: separate
+  int32_t* ready;         // [m-tiles] fused GEMM readiness counters, zeroed by the scan; may be null
   int tiling;             // as set on the plan: 0 (default, = 1), 1, 2 or 3
   int32_t* tok_mt;        // [Tmax] (slab << 24) | row
   int32_t* tok_need;      // [Tmax] contributions this GPU adds to the token
@@ -176,6 +177,8 @@ __device__ void route_scan_body(const RouteParams& p, int T, int* s_warp) {
     // the tiling this call runs (the host launches only its kernels)
     p.info[3] = p.tiling == 0 ? 1 : p.tiling;
   }
+  if (p.ready)
+    for (int i = threadIdx.x; i < base_tiles; i += blockDim.x) p.ready[i] = 0;
 }
 
 // 2 as its own launch (one block of 1024 threads).

@@ -206,14 +206,20 @@ AFD_API afd_status_t afd_ffn_get_kernel_times(afd_ffn_plan_t plan, float* ms);
 /*
  * Tiling of the two grouped GEMMs, chosen on the host for the following calls.
  * 0 (default) or 1: one CTA per 128-row x 256-column tile, A rows from the gather stage's
- * expert-ordered copy.
+ * expert-ordered copy; W13 and W2 are two launches.
  * 2: CTA pairs on 256-row tiles (cta_group::2 MMAs, less operand traffic per MMA, but a
  *    per-K-block handshake between the two SMs that measured about 2x slower).
  * 3: as 1, but the W13 kernel fetches its A rows straight from the slabs with TMA
  *    tile::gather4 (no row copy; 32 four-row requests per A tile, measured about 2.7x
  *    slower for W13 on a 4096-token DeepSeek-V3 share).
- * Results are the same within rounding; tilings 2 and 3 exist for tests and measurements.
- * Returns AFD_ERR_INVALID_ARGUMENT outside 0..3.
+ * 4: as 1, but W13 and W2 run in one persistent launch: every CTA walks its W13 tiles and
+ *    then its W2 tiles; a W2 tile waits (bounded) on a per-m-tile counter that the W13
+ *    epilogues of its m-tile release. Measured slower than two launches on the 4096-token
+ *    DeepSeek-V3 share (1668 against 1446 us) although each half alone runs at its
+ *    two-launch speed.
+ * Results are the same within rounding; tilings 2, 3 and 4 exist for tests and
+ * measurements. afd_ffn_kernels_per_layer counts the default tiling's launches (tiling 4
+ * makes one fewer). Returns AFD_ERR_INVALID_ARGUMENT outside 0..4.
  */
 AFD_API afd_status_t afd_ffn_set_tiling(afd_ffn_plan_t plan, int32_t tiling);
 

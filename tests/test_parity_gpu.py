@@ -41,7 +41,7 @@ def test_random_shapes_several_tiles(seed, shape, counts, cap, zipf):
     assert res["status_rc"] == 0
 
 
-@pytest.mark.parametrize("tiling", [1, 2, 3])
+@pytest.mark.parametrize("tiling", [1, 2, 3, 4])
 @pytest.mark.parametrize("seed,shape,counts,cap", [
     # experts of a few hundred rows: pair tiles whose second CTA is partly or fully empty
     (21, W.LayerShape(512, 256, 4, 0, 4, 1, 2), [300, 217, 0, 65], 300),
@@ -161,6 +161,7 @@ def _sampled_check(name, n_sample=40, tiling=0):
 @pytest.mark.parametrize("name,tiling", [("qwen3_235b_t2048", 0), ("deepseek_v3_share_t4096", 0),
                                          ("deepseek_v3_share_t4096", 2),
                                          ("deepseek_v3_share_t4096", 3),
+                                         ("deepseek_v3_share_t4096", 4),
                                          ("qwen3_235b_spec_q4_t8192", 0)])
 def test_full_size_sampled(name, tiling):
     _sampled_check(name, tiling=tiling)
