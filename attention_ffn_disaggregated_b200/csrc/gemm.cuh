@@ -9,7 +9,7 @@
 // registers ("software promotion": the scales are arbitrary fp32, so they cannot ride on
 // the hardware's UE8M0 block-scale path).
 //
-// Two tilings (the routing scan records which one a call uses; see route_scan_kernel):
+// Tilings (the host launches the kernels of the one set on the plan):
 //   PAIR = 1  one CTA per tile; per K block it loads A 128x128 and B 256x128 (48 KiB).
 //   PAIR = 2  a CTA pair (cluster of two) shares a 256-row tile of one expert: each CTA
 //             loads its own 128 A rows and half of B (32 KiB per K block), the leader
@@ -18,6 +18,8 @@
 //             K block needs a partial-ready / partial-drained handshake between the two
 //             SMs; with only one K block of TMEM slack that latency is exposed, and on
 //             the measured workloads this tiling is about 2x slower. Opt-in only.
+//   GATHER    (W13, PAIR = 1) the A rows come straight from the slabs by tile::gather4.
+//   EPI_FUSED (PAIR = 1) W13 and W2 tiles in one persistent launch (see FusedArgs).
 //
 // Warp roles (384 threads): warp 0 issues TMA loads, warp 1 owns TMEM and (leader) issues
 // MMAs, warps 2..3 idle, warps 4..11 are the epilogue (two per TMEM lane quadrant,
