@@ -55,6 +55,21 @@ def test_both_tilings(tiling, seed, shape, counts, cap):
     assert res["status_rc"] == 0
 
 
+# The ABI's limits in one layer: 1024 groups (1023 local experts + shared), top-K 32 and
+# 128 slabs of two tokens each; every tiling (the slab-gather tiling then carries 128
+# per-slab tensor maps).
+_LIMITS_SHAPE = W.LayerShape(256, 128, 1024, 0, 1023, 1, 32)
+
+
+@pytest.mark.parametrize("tiling", [1, 2, 3, 4])
+def test_limits_groups_topk_slabs(tiling):
+    inp = W.make_custom_inputs(_LIMITS_SHAPE, [2] * 128, 2, seed=31)
+    res, ref, _ = _full_check(inp, calls=1, tiling=tiling)
+    assert res["tiling"] == tiling and res["status_rc"] == 0
+    # id 1023 is not held here, so a token that picked it has 31 local rows + shared
+    assert 256 * 31 < ref["routing"].num_rows <= 256 * 33
+
+
 def test_repeated_calls_self_clean():
     """The combine accumulators are cleared by the last contributor: call twice, same result."""
     inp = W.make_custom_inputs(W.LayerShape(512, 256, 12, 2, 8, 1, 4), [200, 90], 200, seed=7)
