@@ -99,7 +99,8 @@ typedef struct CUstream_st* afd_stream_t; /* same type as cudaStream_t; NULL = l
 typedef struct afd_ffn_plan_s* afd_ffn_plan_t; /* opaque; owned by the library */
 
 typedef struct {
-  int32_t hidden;             /* H, multiple of 128 */
+  int32_t hidden;             /* H, multiple of 128; AFD_ERR_UNSUPPORTED unless a multiple
+                                 of 256 (the down projection writes 256-column tiles) */
   int32_t intermediate;       /* I, multiple of 128 */
   int32_t num_experts_global; /* E_g >= 1: ids the router may emit are [0, E_g) */
   int32_t expert_begin;       /* e0 >= 0 */
