@@ -216,7 +216,7 @@ AFD_API afd_status_t afd_ffn_get_kernel_times(afd_ffn_plan_t plan, float* ms);
  * 4: as 1, but W13 and W2 run in one persistent launch: every CTA walks its W13 tiles and
  *    then its W2 tiles; a W2 tile waits (bounded) on a per-m-tile counter that the W13
  *    epilogues of its m-tile release. Measured slower than two launches on the 4096-token
- *    DeepSeek-V3 share (1668 against 1446 us) although each half alone runs at its
+ *    DeepSeek-V3 share (1582 against 1446 us) although each half alone runs at its
  *    two-launch speed.
  * Results are the same within rounding; tilings 2, 3 and 4 exist for tests and
  * measurements. afd_ffn_kernels_per_layer counts the default tiling's launches (tiling 4
