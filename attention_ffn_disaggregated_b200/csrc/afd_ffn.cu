@@ -309,7 +309,15 @@ afd_status_t afd_ffn_plan(const afd_ffn_config_t* cfg, const afd_ffn_weights_t* 
     delete P;
     return AFD_ERR_CUDA;
   }
-  for (int i = 0; i <= AFD_NUM_KERNELS; ++i) cudaEventCreate(&P->ev[i]);
+  for (int i = 0; i <= AFD_NUM_KERNELS; ++i) {
+    if (cudaEventCreate(&P->ev[i]) != cudaSuccess) {
+      cudaGetLastError();
+      for (int j = 0; j < i; ++j) cudaEventDestroy(P->ev[j]);
+      cudaFree(P->ws);
+      delete P;
+      return AFD_ERR_CUDA;
+    }
+  }
   *out = P;
   return AFD_OK;
 }
@@ -427,6 +435,11 @@ static void fill_gemm_params(afd_ffn_plan_t P, int epi, GemmParams& gp) {
 afd_status_t afd_ffn_layer(afd_ffn_plan_t P, const afd_slab_t* slabs, const int32_t* d_counts,
                            afd_stream_t stream_) {
   if (!P || !slabs || !d_counts) return AFD_ERR_INVALID_ARGUMENT;
+  {
+    // the plan's workspace and tensor maps belong to the device it was built on
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev != P->device) return AFD_ERR_INVALID_ARGUMENT;
+  }
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   const afd_ffn_config_t& c = P->cfg;
   SlabTable tab;

@@ -102,8 +102,17 @@ def check_config(cfg: Config) -> int:
     return lib().afd_ffn_check_config(ctypes.byref(cfg))
 
 
-def _ptr(t) -> Optional[int]:
-    return None if t is None else t.data_ptr()
+def _ptr(t, name: str = "tensor") -> Optional[int]:
+    """Device address of a CUDA tensor (None stays None). The kernels read these addresses
+    as dense device arrays, so host or strided tensors are refused here rather than
+    handed to the GPU."""
+    if t is None:
+        return None
+    if not getattr(t, "is_cuda", False):
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
 
 
 def _stream_handle(stream) -> Optional[int]:
@@ -128,7 +137,8 @@ class FfnLayer:
         self.slab_capacity = slab_capacity
         self._keep = (w13, w13_scale, w2, w2_scale)
         self.cfg = make_config(shape, num_slabs, slab_capacity)
-        w = Weights(_ptr(w13), _ptr(w13_scale), _ptr(w2), _ptr(w2_scale))
+        w = Weights(_ptr(w13, "w13"), _ptr(w13_scale, "w13_scale"), _ptr(w2, "w2"),
+                    _ptr(w2_scale, "w2_scale"))
         h = c_void_p()
         rc = L.afd_ffn_plan(ctypes.byref(self.cfg), ctypes.byref(w), ctypes.byref(h))
         if rc != AFD_OK:
@@ -154,9 +164,10 @@ class FfnLayer:
         if len(slabs) != self.num_slabs:
             raise ValueError("expected %d slabs" % self.num_slabs)
         for i, s in enumerate(slabs):
-            self._descs[i] = SlabDesc(_ptr(s.x), _ptr(s.x_scale), _ptr(s.topk_ids),
-                                      _ptr(s.topk_weights), _ptr(s.y))
-        rc = lib().afd_ffn_layer(self.plan, self._descs, c_void_p(_ptr(counts)),
+            self._descs[i] = SlabDesc(_ptr(s.x, "x"), _ptr(s.x_scale, "x_scale"),
+                                      _ptr(s.topk_ids, "topk_ids"),
+                                      _ptr(s.topk_weights, "topk_weights"), _ptr(s.y, "y"))
+        rc = lib().afd_ffn_layer(self.plan, self._descs, c_void_p(_ptr(counts, "counts")),
                                  c_void_p(_stream_handle(stream)))
         if rc != AFD_OK:
             raise AfdError(rc, "afd_ffn_layer")
@@ -264,9 +275,10 @@ def route_noalloc(shape, slabs: Sequence, counts, stream=None) -> dict:
     }
     descs = (SlabDesc * M)()
     for i, s in enumerate(slabs):
-        descs[i] = SlabDesc(_ptr(s.x), _ptr(s.x_scale), _ptr(s.topk_ids), _ptr(s.topk_weights), _ptr(s.y))
+        descs[i] = SlabDesc(_ptr(s.x, "x"), _ptr(s.x_scale, "x_scale"), _ptr(s.topk_ids, "topk_ids"),
+                            _ptr(s.topk_weights, "topk_weights"), _ptr(s.y, "y"))
     P = lambda k: c_void_p(out[k].data_ptr())
-    rc = lib().afd_ffn_route_noalloc(ctypes.byref(cfg), descs, c_void_p(_ptr(counts)), P("sizes"),
+    rc = lib().afd_ffn_route_noalloc(ctypes.byref(cfg), descs, c_void_p(_ptr(counts, "counts")), P("sizes"),
                                      P("counts"), P("offsets"), P("row_token"), P("row_k"),
                                      P("row_weight"), P("pos"), P("status"),
                                      c_void_p(_stream_handle(stream)))

@@ -157,8 +157,8 @@ AFD_API afd_status_t afd_ffn_plan(const afd_ffn_config_t* cfg, const afd_ffn_wei
  * slabs: host array of num_slabs descriptors (read during the call only; the device
  * buffers they point to must stay valid until the stream reaches the work).
  * d_counts: device int32 [num_slabs]. Returns AFD_ERR_INVALID_ARGUMENT for NULL
- * arguments or misaligned slab pointers (nothing enqueued) and AFD_ERR_CUDA if a
- * launch fails.
+ * arguments, misaligned slab pointers or a current CUDA device other than the plan's
+ * (nothing enqueued) and AFD_ERR_CUDA if a launch fails.
  */
 AFD_API afd_status_t afd_ffn_layer(afd_ffn_plan_t plan, const afd_slab_t* slabs, const int32_t* d_counts,
                            afd_stream_t stream);

@@ -104,3 +104,13 @@ def test_plan_without_gpu_is_unsupported():
     h = ctypes.c_void_p()
     assert L.afd_ffn_plan(ctypes.byref(c), ctypes.byref(w), ctypes.byref(h)) == 2
     assert h.value is None
+
+
+def test_binding_refuses_host_tensors():
+    """The binding hands only CUDA tensors' addresses to the library: a host tensor
+    (which the kernels would read as a device address) is refused before any call."""
+    import torch
+    from attention_ffn_disaggregated_b200.ffn import _ptr
+    assert _ptr(None) is None
+    with pytest.raises(ValueError, match="w13 must be a CUDA tensor"):
+        _ptr(torch.zeros(16, dtype=torch.uint8), "w13")
