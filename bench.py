@@ -474,6 +474,20 @@ def main():
     if rc != 0:
         raise RuntimeError(f"layer status {rc} word {word:#x} after timing")
 
+    # for context: the same call replayed from a CUDA graph (the direct-launch time above
+    # stays the reported value)
+    graph_ms = None
+    if not args.graph:
+        gms = time_layer(layer, slabs, counts, flush, min(args.steps, 10), 2, graph=True)
+        graph_ms = float(np.mean(gms))
+        if world > 1:
+            t = torch.tensor([graph_ms], device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            graph_ms = float(t.item())
+        rc, word = layer.status()
+        if rc != 0:
+            raise RuntimeError(f"layer status {rc} word {word:#x} after the graph replays")
+
     # end to end through the public API from pinned host memory (uploads, layer and
     # downloads inside the timed region), serial and two-deep pipelined
     layer.set_timing(False)
@@ -547,6 +561,7 @@ def main():
                                "frac": t_roof * 1e3 / layer_ms, "alg_bytes": bytes_alg,
                                "alg_flops": flops_alg, "hbm_gbs": hbm, "fp8_tflops": fp8_peak},
             "kernel_ms": stage_ms,
+            "graph_replay_ms_per_step": graph_ms,
             "routed_rows_per_s": world * args.steps * R / (tot_ms * 1e-3),
             "e2e": {"value": world * T / (e2e_pipe_ms * 1e-3), "unit": "tokens/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
