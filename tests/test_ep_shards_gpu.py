@@ -1,0 +1,45 @@
+"""Expert-parallel sharding on the GPU path: two FFN shards over the same slabs.
+
+An FFN pool shards the experts: each GPU holds a disjoint id range [e0, e0 + E_l), skips
+the ids it does not hold, and returns a partial sum that the attention side adds up (the
+M2N push-back). Here both shards run on one GPU, as two plans with the same slabs: shard
+A holds experts 0..7 and the shared expert, shard B experts 8..15. The sum of their bf16
+partial outputs must match the oracle's full layer (all 16 experts + shared) within the
+row tolerance; each partial must also match the oracle run on its own shard.
+"""
+import numpy as np
+import pytest
+
+import workloads as W
+from oracle import ffn as offn
+from oracle import fp8 as ofp8
+from tests.helpers import TOL_ROW_RMS, compare_outputs, run_cuda_layer
+
+pytestmark = pytest.mark.gpu
+
+
+def _shard(full, shape, lo, hi, with_shared):
+    """The full model's inputs restricted to the weights of experts [lo, hi) (+ shared)."""
+    idx = list(range(lo, hi)) + ([full.shape.num_local_experts] if with_shared else [])
+    return W.LayerInputs(shape, full.w13[idx], full.w13_scale[idx], full.w2[idx], full.w2_scale[idx],
+                         full.slabs, full.counts, full.capacity)
+
+
+@pytest.mark.parametrize("counts,cap,zipf", [([200, 37, 0, 129], 200, None), ([512, 300], 512, 1.0)])
+def test_two_expert_shards_sum_to_the_full_layer(counts, cap, zipf):
+    H, I, Eg, K = 512, 256, 16, 4
+    full = W.make_custom_inputs(W.LayerShape(H, I, Eg, 0, Eg, 1, K), counts, cap, seed=41, zipf_s=zipf)
+    a = _shard(full, W.LayerShape(H, I, Eg, 0, 8, 1, K), 0, 8, True)
+    b = _shard(full, W.LayerShape(H, I, Eg, 8, 8, 0, K), 8, 16, False)
+    ref = offn.ffn_layer(full)["out"]
+    parts = []
+    for shard in (a, b):
+        res = run_cuda_layer(shard)
+        assert res["status_rc"] == 0
+        compare_outputs(res["outs"][0], offn.ffn_layer(shard)["out"])
+        parts.append(ofp8.bf16_from_bits(res["outs"][0]))
+    total = parts[0] + parts[1]
+    rms = np.sqrt((ref ** 2).mean(axis=1))
+    err = np.abs(total - ref).max(axis=1)
+    # two bf16 roundings instead of one: the same row tolerance still holds comfortably
+    assert np.all(err <= TOL_ROW_RMS * rms), float((err / rms).max())
