@@ -6,6 +6,7 @@ contribution must be exactly zero. Sizes here span several 128-row and 256-colum
 with ragged tails; the full-size workloads are checked on sampled tokens.
 """
 import numpy as np
+import torch
 import pytest
 
 import workloads as W
@@ -180,3 +181,21 @@ def _sampled_check(name, n_sample=40, tiling=0):
                                          ("qwen3_235b_spec_q4_t8192", 0)])
 def test_full_size_sampled(name, tiling):
     _sampled_check(name, tiling=tiling)
+
+
+# --------------------------------------------------------------- sweep cells (T x M)
+
+@pytest.fixture(scope="module")
+def share_weights():
+    """One weight set of the DeepSeek-V3 share shape for the sweep cells (as bench.py's
+    sweep uses), generated once for the module."""
+    return W.make_weights(W.DEEPSEEK_V3_SHARE, torch.Generator().manual_seed(4))
+
+
+@pytest.mark.parametrize("cell", ["sweep_t1_m64_uniform", "sweep_t8_m16_zipf1.2", "sweep_t64_m4_uniform"])
+def test_sweep_cells_full_parity(cell, share_weights):
+    """Small-batch cells of the T x M sweep, every output row against the oracle: a single
+    token among 64 slabs (63 empty), a few skewed tokens, and 64 tokens over 4 slabs."""
+    inp = W.make_inputs(W.workload_by_name(cell), weights=share_weights)
+    res, _, _ = _full_check(inp)
+    assert res["status_rc"] == 0
