@@ -443,6 +443,9 @@ def main():
             # separate pass of directly launched calls below
             step_ms = time_layer(layer, slabs, counts, flush, args.steps, 0, graph=True)
         else:
+            # per-kernel events stay off in the timed calls (they would sit between the
+            # layer's launches); stage times come from a separate pass below
+            layer.set_timing(False)
             for _ in range(args.steps):
                 flush.zero_()
                 e0 = torch.cuda.Event(enable_timing=True)
@@ -452,15 +455,14 @@ def main():
                 e1.record(stream)
                 e1.synchronize()
                 step_ms.append(e0.elapsed_time(e1))
-                for k, v in layer.kernel_times().items():
-                    kt[k].append(v)
-    if args.graph:
-        for _ in range(min(args.steps, 5)):
-            flush.zero_()
-            layer(slabs, counts)
-            torch.cuda.synchronize()
-            for k, v in layer.kernel_times().items():
-                kt[k].append(v)
+            layer.set_timing(True)
+    # stage times: a few further calls with per-kernel events (not part of the timed steps)
+    for _ in range(min(args.steps, 5)):
+        flush.zero_()
+        layer(slabs, counts)
+        torch.cuda.synchronize()
+        for k, v in layer.kernel_times().items():
+            kt[k].append(v)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
