@@ -207,7 +207,12 @@ def run_reference(args):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * tot / len(times), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": wl.name, "tokens": T, "slabs": wl.num_slabs},
+        "config": {"workload": wl.name, "tokens": T, "slabs": wl.num_slabs,
+                   "hidden": wl.shape.hidden, "intermediate": wl.shape.intermediate,
+                   "local_experts": wl.shape.num_local_experts,
+                   "shared_expert": wl.shape.has_shared_expert, "top_k": wl.shape.top_k,
+                   "routed_rows": int(rt.num_rows), "active_experts": int(np.sum(rt.counts > 0)),
+                   "parallelism": "replica x1"},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": os.cpu_count(), "kind": "oracle",
                          "sample": f"{per_step} tokens per step of the {T}-token workload"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
