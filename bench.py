@@ -88,8 +88,9 @@ def source_hash():
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(kernel: str):
-    """DRAM bytes per launch recorded by ncu for this kernel source (None if stale/missing)."""
+def profiled_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch recorded by ncu for this kernel source on this workload (None
+    if stale, missing or captured on another workload)."""
     p = os.path.join(ROOT, "profiles", f"{kernel}_traffic.txt")
     if not os.path.exists(p):
         return None
@@ -98,7 +99,7 @@ def profiled_traffic(kernel: str):
         if ":" in line and not line.startswith("#"):
             k, v = line.split(":", 1)
             kv[k.strip()] = v.strip()
-    if kv.get("source_sha") != source_hash():
+    if kv.get("source_sha") != source_hash() or kv.get("workload") != workload:
         return None
     try:
         return float(kv["dram_bytes_per_launch_full"])
@@ -562,7 +563,7 @@ def main():
                        "parallelism": f"replica x{world}"},
             "roofline": {"bound": "tensor", "kernel": dominant, "achieved": achieved,
                          "peak": fp8_peak, "unit": "TFLOP/s", "frac": achieved / fp8_peak,
-                         "traffic": profiled_traffic(dominant),
+                         "traffic": profiled_traffic(dominant, wl.name),
                          "peak_source": f"{peak_src} bf16 burst x 2 (fp8/bf16 nominal ratio)"},
             "layer_roofline": {"bound": bound, "t_roof_ms": t_roof * 1e3, "t_layer_ms": layer_ms,
                                "frac": t_roof * 1e3 / layer_ms, "alg_bytes": bytes_alg,
