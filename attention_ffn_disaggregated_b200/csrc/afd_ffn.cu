@@ -20,6 +20,7 @@
 
 #include "afd_ffn.h"
 #include "gemm.cuh"
+#include "gemm_mx.cuh"
 #include "route.cuh"
 
 using namespace afd;
@@ -63,6 +64,10 @@ struct afd_ffn_plan_s {
   int* status;
   int* scan_ticket;   // route_count's last-block counter, zero between calls
   int32_t* ready;     // fused W13->W2 launch: per m-tile readiness counters
+  // tiling 5 (block-scale W13): factor images of the activation rows (workspace) and of
+  // W13 (allocated and built when the tiling is first selected)
+  uint8_t* mx_sfa;
+  uint8_t* mx_sfb = nullptr;
   CUtensorMap tm_a13, tm_w13, tm_a2, tm_w2;
   // tiling 3 (W13 rows gathered from the slabs): one map per slab, re-encoded when a slab's
   // row pointer changes between calls
@@ -179,7 +184,8 @@ afd_status_t afd_ffn_plan(const afd_ffn_config_t* cfg, const afd_ffn_weights_t* 
   // The GEMM kernels split the block's registers between warpgroups with setmaxnreg; that
   // is only safe when the block is launched with exactly the budget the split assumes.
   {
-    const void* fns[6] = {reinterpret_cast<const void*>(grouped_gemm_kernel<EPI_FUSED, 1, false>),
+    const void* fns[7] = {reinterpret_cast<const void*>(grouped_gemm_kernel<EPI_FUSED, 1, false>),
+                          reinterpret_cast<const void*>(w13_mx_kernel),
                           reinterpret_cast<const void*>(grouped_gemm_kernel<EPI_SWIGLU, 1, false>),
                           reinterpret_cast<const void*>(grouped_gemm_kernel<EPI_SWIGLU, 1, true>),
                           reinterpret_cast<const void*>(grouped_gemm_kernel<EPI_SWIGLU, 2, false>),
@@ -238,6 +244,7 @@ afd_status_t afd_ffn_plan(const afd_ffn_config_t* cfg, const afd_ffn_weights_t* 
   const size_t o_hq = take(static_cast<size_t>(P->rpad) * I, 1024);
   const size_t o_sh_t = take(sizeof(float) * static_cast<size_t>(I / 128) * P->rpad, 256);
   const size_t o_acc = take(sizeof(float) * static_cast<size_t>(P->Tmax) * H, 256);
+  const size_t o_mx_sfa = take(static_cast<size_t>(P->rpad / 128 + P->G) * (H / 128) * kSfImage, 256);
   P->ws_bytes = take(0, 256);
 
   if (cudaMalloc(&P->ws, P->ws_bytes) != cudaSuccess) {
@@ -273,6 +280,7 @@ afd_status_t afd_ffn_plan(const afd_ffn_config_t* cfg, const afd_ffn_weights_t* 
   P->hq = b + o_hq;
   P->sh_t = reinterpret_cast<float*>(b + o_sh_t);
   P->acc = reinterpret_cast<float*>(b + o_acc);
+  P->mx_sfa = b + o_mx_sfa;
 
   const int E = P->G;
   st = encode_2d(enc, &P->tm_a13, P->a_perm, H, P->rpad);
@@ -288,6 +296,8 @@ afd_status_t afd_ffn_plan(const afd_ffn_config_t* cfg, const afd_ffn_weights_t* 
   P->scatter_smem = sizeof(int32_t) * (static_cast<size_t>(kRouteWarps) * El1 + kRouteWarps * 32 * K);
   if (cudaFuncSetAttribute(grouped_gemm_kernel<EPI_FUSED, 1, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(gemm_smem_bytes(EPI_FUSED))) != cudaSuccess ||
+      cudaFuncSetAttribute(w13_mx_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(mx_smem_bytes())) != cudaSuccess ||
       cudaFuncSetAttribute(grouped_gemm_kernel<EPI_SWIGLU, 1, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(gemm_smem_bytes(EPI_SWIGLU))) != cudaSuccess ||
       cudaFuncSetAttribute(grouped_gemm_kernel<EPI_SWIGLU, 1, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -328,6 +338,7 @@ void afd_ffn_destroy(afd_ffn_plan_t P) {
   for (int i = 0; i <= AFD_NUM_KERNELS; ++i)
     if (P->ev[i]) cudaEventDestroy(P->ev[i]);
   if (P->ws) cudaFree(P->ws);
+  if (P->mx_sfb) cudaFree(P->mx_sfb);
   delete P;
 }
 
@@ -463,7 +474,7 @@ afd_status_t afd_ffn_layer(afd_ffn_plan_t P, const afd_slab_t* slabs, const int3
   // expert-ordered copy of the rows made by the gather stage; tiling 3 gathers them from
   // the slabs inside the W13 kernel (tile::gather4)
   const int tiling = P->tiling == 0 ? 1 : P->tiling;
-  const bool pair = tiling == 2, slab_gather = tiling == 3, fused = tiling == 4;
+  const bool pair = tiling == 2, slab_gather = tiling == 3, fused = tiling == 4, mx = tiling == 5;
   if (slab_gather) {
     EncodeTiledFn enc = get_encode_fn();
     if (!enc) return AFD_ERR_CUDA;
@@ -505,6 +516,13 @@ afd_status_t afd_ffn_layer(afd_ffn_plan_t P, const afd_slab_t* slabs, const int3
     fa.ready = P->ready;
     grouped_gemm_kernel<EPI_FUSED, 1, false><<<grid1, kGemmThreads, gemm_smem_bytes(EPI_FUSED), stream>>>(
         g13, P->tm_a13, P->tm_w13, ytab, fa);
+  } else if (mx) {
+    // factor images of this call's activation rows, then W13 on the block-scale path (the
+    // W13 stage time includes the image kernel)
+    mx_act_sf_kernel<<<P->num_sms * 4, 128, 0, stream>>>(P->mtile_off, P->group_off, P->G, P->sa_t,
+                                                         P->rpad, c.hidden / 128, P->mx_sfa, P->status);
+    w13_mx_kernel<<<grid1, kGemmThreads, mx_smem_bytes(), stream>>>(g13, P->tm_a13, P->tm_w13,
+                                                                   MxArgs{P->mx_sfa, P->mx_sfb});
   } else if (slab_gather) {
     grouped_gemm_kernel<EPI_SWIGLU, 1, true><<<grid1, kGemmThreads, gemm_smem_bytes(EPI_SWIGLU), stream>>>(
         g13, P->tm_a13, P->tm_w13, ytab, P->slab_maps);
@@ -541,6 +559,7 @@ afd_status_t afd_ffn_get_status(afd_ffn_plan_t P, afd_stream_t stream, int32_t* 
   if (word) *word = v;
   if (v & AFD_STATUS_TIMEOUT) return AFD_ERR_TIMEOUT;
   if (v & (AFD_STATUS_BAD_ROUTING | AFD_STATUS_BAD_COUNT)) return AFD_ERR_BAD_ROUTING;
+  if (v & AFD_STATUS_BAD_SCALE) return AFD_ERR_INVALID_ARGUMENT;
   return AFD_OK;
 }
 
@@ -616,7 +635,26 @@ afd_status_t afd_ffn_set_wait_limit(afd_ffn_plan_t P, int64_t limit_ns) {
 }
 
 afd_status_t afd_ffn_set_tiling(afd_ffn_plan_t P, int32_t tiling) {
-  if (!P || tiling < 0 || tiling > 4) return AFD_ERR_INVALID_ARGUMENT;
+  if (!P || tiling < 0 || tiling > 5) return AFD_ERR_INVALID_ARGUMENT;
+  if (tiling == 5 && !P->mx_sfb) {
+    // the W13 factor images, once per plan (the weights are fixed for its lifetime)
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev != P->device) return AFD_ERR_INVALID_ARGUMENT;
+    const afd_ffn_config_t& c = P->cfg;
+    const size_t n_img = static_cast<size_t>(P->G) * (2 * c.intermediate / 128) * (c.hidden / 128);
+    if (n_img >= (size_t{1} << 31)) return AFD_ERR_UNSUPPORTED;
+    uint8_t* img = nullptr;
+    if (cudaMalloc(&img, n_img * kSfImage) != cudaSuccess) {
+      cudaGetLastError();
+      return AFD_ERR_OUT_OF_MEMORY;
+    }
+    mx_weight_sf_kernel<<<P->num_sms * 4, 256>>>(P->w.w13_scale, static_cast<int>(n_img), img, P->status);
+    if (cudaGetLastError() != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
+      cudaFree(img);
+      return AFD_ERR_CUDA;
+    }
+    P->mx_sfb = img;
+  }
   P->tiling = tiling;
   return AFD_OK;
 }

@@ -212,6 +212,55 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
       : "memory");
 }
 
+// Block-scaled form, kind::mxf8f6f4 with UE8M0 factors (2^(byte - 127)) read from TMEM:
+// one factor per 32 K elements for each row of A (at `sfa`) and each column of B (at
+// `sfb`). Instruction descriptor: A and B e4m3 (bits 7-9, 10-12 = 0), both K-major,
+// N >> 3 at bits 17-22, factor type UE8M0 (bit 23), M >> 4 at bits 24-28; the factor byte
+// ids (bits 4-5 for B, 29-30 for A) are 0, and K is 32 per instruction (bit 31 = 0).
+__host__ __device__ constexpr uint32_t idesc_mx_e4m3(int M, int N) {
+  return (static_cast<uint32_t>(N >> 3) << 17) | (1u << 23) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma_mx_e4m3(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                             uint32_t idesc, uint32_t sfa, uint32_t sfb,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+          d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+
+// Shared memory -> TMEM: 32 rows of 16 bytes, row i to lane i of four consecutive 32-bit
+// columns, written into all four lane quadrants. Executes in order with the issuing
+// thread's MMAs.
+__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+// Descriptor of such a source block: 16-byte rows stored one after another without
+// swizzling (layout type 0), so 8-row groups are 128 bytes apart (stride byte offset);
+// the leading byte offset is unused for a single 16-byte column.
+__device__ __forceinline__ uint64_t sdesc_rows16(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>(128u >> 4) << 32;
+  d |= static_cast<uint64_t>(1u) << 46;
+  return d;
+}
+
+// Plain bulk copy, global -> this CTA's shared memory (no multicast), completing `bytes`
+// on `bar`. Both addresses 16-byte aligned, `bytes` a multiple of 16.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
 // 32 lanes x 32 consecutive 32-bit columns: thread i of the warp receives row
 // (warp's lane quadrant base + i), columns [col, col + 32).
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {

@@ -42,7 +42,7 @@ struct RouteParams {
   int32_t* mtile2_off;    // [G+1] 256-row m-tiles (CTA-pair tiling); may be null
   int* scan_ticket;       // zero between calls: route_count runs the scan; null: separate
   int32_t* ready;         // [m-tiles] fused GEMM readiness counters, zeroed by the scan; may be null
-  int tiling;             // as set on the plan: 0 (default, = 1), 1, 2 or 3
+  int tiling;             // as set on the plan: 0 (default, = 1) .. 5
   int32_t* tok_mt;        // [Tmax] (slab << 24) | row
   int32_t* tok_need;      // [Tmax] contributions this GPU adds to the token
   int32_t* pos;           // [Tmax*K]

@@ -20,7 +20,7 @@ AFD_OK = 0
 STATUS_NAMES = {0: "AFD_OK", 1: "AFD_ERR_INVALID_ARGUMENT", 2: "AFD_ERR_UNSUPPORTED",
                 3: "AFD_ERR_OUT_OF_MEMORY", 4: "AFD_ERR_CUDA", 5: "AFD_ERR_BAD_ROUTING",
                 6: "AFD_ERR_TIMEOUT"}
-STATUS_BAD_ROUTING, STATUS_TIMEOUT, STATUS_BAD_COUNT = 0x1, 0x2, 0x4
+STATUS_BAD_ROUTING, STATUS_TIMEOUT, STATUS_BAD_COUNT, STATUS_BAD_SCALE = 0x1, 0x2, 0x4, 0x8
 KERNEL_NAMES = ["route_count", "route_scan", "route_scatter", "gather_rows", "gemm13_swiglu",
                 "gemm2_combine", "combine_finalize"]
 
@@ -228,13 +228,16 @@ class FfnLayer:
 
     def set_tiling(self, tiling: int):
         """0: default (1); 1: single-CTA tiles; 2: CTA-pair tiles; 3: single-CTA tiles with the
-        W13 rows gathered from the slabs by TMA (no expert-ordered row copy)."""
+        W13 rows gathered from the slabs by TMA (no expert-ordered row copy); 4: W13 and W2 in
+        one persistent launch; 5: W13 on the block-scale MMA path, for inputs whose
+        activation and W13 block scales are all powers of two (the first selection builds
+        the W13 factor images and synchronises the device)."""
         rc = lib().afd_ffn_set_tiling(self.plan, int(tiling))
         if rc != AFD_OK:
             raise AfdError(rc, "afd_ffn_set_tiling")
 
     def tiling(self, stream=None) -> int:
-        """Tiling (1 or 2) the last layer call used."""
+        """Tiling (1 to 5) the last layer call used."""
         t = c_int32(0)
         rc = lib().afd_ffn_get_tiling(self.plan, c_void_p(_stream_handle(stream)), ctypes.byref(t))
         if rc != AFD_OK:

@@ -15,6 +15,7 @@ scaling is weak and value = all ranks' tokens / max over ranks of the device tim
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import os
@@ -44,7 +45,7 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-tokens", type=int, default=64)
-    ap.add_argument("--tiling", type=int, default=0, choices=[0, 1, 2, 3, 4],
+    ap.add_argument("--tiling", type=int, default=0, choices=[0, 1, 2, 3, 4, 5],
                     help="GEMM tiling (afd_ffn_set_tiling); 0 = the library default")
     ap.add_argument("--graph", action="store_true",
                     help="time replays of the layer captured in a CUDA graph")
@@ -407,12 +408,11 @@ def main():
                                 device_id=torch.device("cuda", local))
 
     base = W.workload_by_name(args.config)
-    wl = W.Workload(base.name, base.shape, base.num_tokens, base.num_slabs, base.zipf_s,
-                    base.zero_pop_mod, seed=tuple(base.seed) if rank == 0 else (base.seed[0], 1000 + rank))
+    wl = dataclasses.replace(base, seed=tuple(base.seed) if rank == 0 else (base.seed[0], 1000 + rank))
     weights = None
     if rank != 0:
         weights = W.make_weights(wl.shape, __import__("torch").Generator().manual_seed(
-            int(np.random.SeedSequence(list(base.seed)).generate_state(1)[0])))
+            int(np.random.SeedSequence(list(base.seed)).generate_state(1)[0])), base.pow2_scales)
     inp = W.make_inputs(wl, weights=weights)
     T = int(np.sum(inp.counts))
     dev_w = to_device_weights(inp)
@@ -557,7 +557,9 @@ def main():
                        "gemm_tiling": {1: "one CTA per 128x256 tile, W13 and W2 as two launches",
                                        4: "one CTA per 128x256 tile, W13 and W2 in one persistent launch",
                                        2: "CTA pairs on 256x256 tiles (cta_group::2)",
-                                       3: "one CTA per 128x256 tile, W13 rows by tile::gather4"}[tiling],
+                                       3: "one CTA per 128x256 tile, W13 rows by tile::gather4",
+                                       5: "one CTA per 128x256 tile, W13 on the block-scale MMA path "
+                                          "(power-of-two scales), W2 as two-launch"}[tiling],
                        "l2": "flushed between steps (256 MiB write, untimed)",
                        "launch": "CUDA graph replay" if args.graph else "direct launches",
                        "parallelism": f"replica x{world}"},
@@ -577,7 +579,7 @@ def main():
                     "mode": "two-deep pipeline: upload of step i+1 and download of step i-1 on "
                             "copy streams during step i; L2 flush before each layer call, timed",
                     "serial": {"value": world * T / (e2e_serial_ms * 1e-3), "ms_per_step": e2e_serial_ms}},
-            "gpu_launches": kernels_per_layer() * args.steps,
+            "gpu_launches": (kernels_per_layer() + {4: -1, 5: 1}.get(tiling, 0)) * args.steps,
             "clocks": clk.summary(),
             "cpu_baseline": cpu,
         }

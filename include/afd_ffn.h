@@ -71,6 +71,8 @@ typedef enum {
 #define AFD_STATUS_BAD_ROUTING 0x1 /* id outside [0, E_g) and != -1, or repeated in a token */
 #define AFD_STATUS_TIMEOUT 0x2     /* a bounded device wait expired; outputs are invalid */
 #define AFD_STATUS_BAD_COUNT 0x4   /* some counts[m] < 0 or > slab_capacity; clamped */
+#define AFD_STATUS_BAD_SCALE 0x8   /* tiling 5: a block scale it read is not a positive normal
+                                      power of two; outputs are invalid */
 
 /* Limits. */
 #define AFD_MAX_SLABS 128
@@ -172,7 +174,8 @@ AFD_API afd_status_t afd_ffn_get_info(afd_ffn_plan_t plan, afd_ffn_plan_info_t* 
 /*
  * Synchronise `stream`, read the device status word into *status_word (may be NULL),
  * and clear it. Returns AFD_ERR_TIMEOUT if the TIMEOUT bit was set, else
- * AFD_ERR_BAD_ROUTING if BAD_ROUTING or BAD_COUNT was set, else AFD_OK.
+ * AFD_ERR_BAD_ROUTING if BAD_ROUTING or BAD_COUNT was set, else AFD_ERR_INVALID_ARGUMENT
+ * if BAD_SCALE was set, else AFD_OK.
  */
 AFD_API afd_status_t afd_ffn_get_status(afd_ffn_plan_t plan, afd_stream_t stream, int32_t* status_word);
 
@@ -218,9 +221,18 @@ AFD_API afd_status_t afd_ffn_get_kernel_times(afd_ffn_plan_t plan, float* ms);
  *    epilogues of its m-tile release. Measured slower than two launches on the 4096-token
  *    DeepSeek-V3 share (1582 against 1446 us) although each half alone runs at its
  *    two-launch speed.
- * Results are the same within rounding; tilings 2, 3 and 4 exist for tests and
+ * 5: as 1, but W13 runs on the tensor core's block-scale path (kind::mxf8f6f4 with UE8M0
+ *    factors): TMEM accumulates a tile's whole K loop and the epilogue runs once per
+ *    tile. Only for inputs whose activation and W13 block scales are all positive normal
+ *    powers of two (each is then exactly its UE8M0 factor); any other scale sets
+ *    AFD_STATUS_BAD_SCALE and afd_ffn_get_status then returns AFD_ERR_INVALID_ARGUMENT.
+ *    The first selection on a plan allocates the W13 factor images (E * 2I/128 * H/128 *
+ *    512 bytes) and builds them with one kernel launch and a device synchronisation
+ *    (AFD_ERR_OUT_OF_MEMORY / AFD_ERR_CUDA on failure; call it on the plan's device).
+ *    Each layer call then adds one launch (the activation factor images).
+ * Results are the same within rounding; tilings 2, 3, 4 and 5 exist for tests and
  * measurements. afd_ffn_kernels_per_layer counts the default tiling's launches (tiling 4
- * makes one fewer). Returns AFD_ERR_INVALID_ARGUMENT outside 0..4.
+ * makes one fewer, tiling 5 one more). Returns AFD_ERR_INVALID_ARGUMENT outside 0..5.
  */
 AFD_API afd_status_t afd_ffn_set_tiling(afd_ffn_plan_t plan, int32_t tiling);
 

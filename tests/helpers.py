@@ -15,7 +15,8 @@ def run_cuda_layer(inp, calls: int = 1, layer=None, tiling: int = 0):
     """Plan (unless given), run `calls` times on the current stream, return outputs/routing.
     tiling: 0 = default (1), 1 = single-CTA tiles, W13 and W2 as two launches, 2 = CTA-pair
     tiles, 3 = single-CTA tiles with the W13 rows gathered from the slabs, 4 = single-CTA
-    tiles, W13 and W2 in one persistent launch."""
+    tiles, W13 and W2 in one persistent launch, 5 = W13 on the block-scale MMA path
+    (power-of-two scales only)."""
     import torch
     from attention_ffn_disaggregated_b200 import FfnLayer
     from attention_ffn_disaggregated_b200.device import (gather_outputs, to_device_counts,

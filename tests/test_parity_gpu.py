@@ -71,6 +71,36 @@ def test_limits_groups_topk_slabs(tiling):
     assert 256 * 31 < ref["routing"].num_rows <= 256 * 33
 
 
+# Tiling 5: W13 on the block-scale MMA path, for power-of-two block scales. The oracle is
+# the same; only the inputs' scales are rounded up to powers of two.
+@pytest.mark.parametrize("seed,shape,counts,cap", [
+    (21, W.LayerShape(512, 256, 4, 0, 4, 1, 2), [300, 217, 0, 65], 300),
+    (22, W.LayerShape(768, 384, 6, 0, 6, 0, 3), [511, 2], 511),
+    (23, W.LayerShape(1024, 256, 16, 4, 6, 1, 4), [1, 0, 130], 130),
+    (24, W.LayerShape(1024, 512, 8, 0, 8, 1, 2), [1000], 1000),
+])
+def test_block_scale_tiling(seed, shape, counts, cap):
+    inp = W.make_custom_inputs(shape, counts, cap, seed=seed, zipf_s=1.0, pow2_scales=True)
+    res, _, _ = _full_check(inp, calls=2, tiling=5)
+    assert res["tiling"] == 5
+    assert res["status_rc"] == 0
+
+
+def test_block_scale_tiling_limits():
+    inp = W.make_custom_inputs(_LIMITS_SHAPE, [2] * 128, 2, seed=31, pow2_scales=True)
+    res, _, _ = _full_check(inp, calls=1, tiling=5)
+    assert res["tiling"] == 5 and res["status_rc"] == 0
+
+
+def test_block_scale_tiling_flags_other_scales():
+    """amax/448 scales are not powers of two: tiling 5 must flag them (the outputs are then
+    invalid; nothing faults)."""
+    from attention_ffn_disaggregated_b200.ffn import STATUS_BAD_SCALE
+    inp = W.make_inputs(W.CONFIGS["tiny"])
+    res = run_cuda_layer(inp, tiling=5)
+    assert res["status_rc"] == 1 and res["status_word"] & STATUS_BAD_SCALE
+
+
 def test_repeated_calls_self_clean():
     """The combine accumulators are cleared by the last contributor: call twice, same result."""
     inp = W.make_custom_inputs(W.LayerShape(512, 256, 12, 2, 8, 1, 4), [200, 90], 200, seed=7)
@@ -178,6 +208,8 @@ def _sampled_check(name, n_sample=40, tiling=0):
                                          ("deepseek_v3_share_t4096", 2),
                                          ("deepseek_v3_share_t4096", 3),
                                          ("deepseek_v3_share_t4096", 4),
+                                         ("deepseek_v3_share_t4096_pow2", 0),
+                                         ("deepseek_v3_share_t4096_pow2", 5),
                                          ("qwen3_235b_spec_q4_t8192", 0)])
 def test_full_size_sampled(name, tiling):
     _sampled_check(name, tiling=tiling)

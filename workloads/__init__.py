@@ -10,6 +10,9 @@ Recipe (readings the pages leave open are stated here and in the design notes):
     e4m3fn with one fp32 scale per 128x128 block (scale = block amax / 448);
   * activations: N(0, 1), quantised to e4m3fn with one fp32 scale per token per
     128 channels;
+  * power-of-two variant (workloads named *_pow2, `pow2_scales=True`): every block scale
+    is amax / 448 rounded up to a power of two (an 8-bit exponent, as FP8 recipes with
+    UE8M0 scales quantise); the codes are then taken against that scale;
   * routing: K distinct expert ids per token, drawn without replacement with
     probability proportional to a popularity vector (Gumbel-top-k on log-popularity);
     uniform = equal popularity, Zipf(s) = popularity of id i proportional to 1/(i+1)^s;
@@ -61,6 +64,7 @@ class Workload:
     zipf_s: Optional[float]    # None = uniform popularity
     zero_pop_mod: Optional[int] = None   # ids with id % mod == mod-1 get popularity 0
     seed: Sequence[int] = (0, 0)
+    pow2_scales: bool = False  # block scales rounded up to powers of two
 
     @property
     def slab_counts(self) -> List[int]:
@@ -83,6 +87,10 @@ CONFIGS = {
                                         seed=(2, 0)),
     "qwen3_235b_spec_q4_t8192": Workload("qwen3_235b_spec_q4_t8192", QWEN3_235B, 8192, 32, 0.8,
                                          zero_pop_mod=16, seed=(3, 0)),
+    # the same draws with power-of-two block scales
+    "tiny_pow2": Workload("tiny_pow2", TINY, 64, 2, None, seed=(0, 0), pow2_scales=True),
+    "deepseek_v3_share_t4096_pow2": Workload("deepseek_v3_share_t4096_pow2", DEEPSEEK_V3_SHARE,
+                                             4096, 16, 1.0, seed=(2, 0), pow2_scales=True),
 }
 
 
@@ -113,26 +121,34 @@ def workload_by_name(name: str) -> Workload:
 # quantisation of inputs (library cast; the layer's own requantisation lives elsewhere)
 # ----------------------------------------------------------------------------------------
 
-def _quant_blocks(x: torch.Tensor, rb: int, cb: int):
+def _pow2_ceil(s: torch.Tensor) -> torch.Tensor:
+    """Smallest power of two >= s (s > 0), exactly: s = m * 2^e with m in [0.5, 1)."""
+    m, e = torch.frexp(s)
+    return torch.ldexp(torch.ones_like(s), torch.where(m == 0.5, e - 1, e))
+
+
+def _quant_blocks(x: torch.Tensor, rb: int, cb: int, pow2: bool = False):
     """Quantise a 2-D fp32 tensor to e4m3fn codes with one scale per (rb x cb) block."""
     R, C = x.shape
     assert R % rb == 0 and C % cb == 0
     xb = x.reshape(R // rb, rb, C // cb, cb)
     amax = xb.abs().amax(dim=(1, 3))
     scale = torch.where(amax > 0, amax / E4M3_MAX, torch.ones_like(amax))
+    if pow2:
+        scale = _pow2_ceil(scale)
     q = (xb / scale[:, None, :, None]).clamp_(-E4M3_MAX, E4M3_MAX)
     codes = q.to(torch.float8_e4m3fn).view(torch.uint8).reshape(R, C)
     return codes, scale.to(torch.float32)
 
 
-def quantise_weight(w: torch.Tensor):
+def quantise_weight(w: torch.Tensor, pow2: bool = False):
     """[N, C] fp32 -> (uint8 codes [N, C], fp32 scales [N/128, C/128])."""
-    return _quant_blocks(w, QBLOCK, QBLOCK)
+    return _quant_blocks(w, QBLOCK, QBLOCK, pow2)
 
 
-def quantise_activation(x: torch.Tensor):
+def quantise_activation(x: torch.Tensor, pow2: bool = False):
     """[n, C] fp32 -> (uint8 codes [n, C], fp32 scales [n, C/128])."""
-    return _quant_blocks(x, 1, QBLOCK)
+    return _quant_blocks(x, 1, QBLOCK, pow2)
 
 
 @dataclasses.dataclass
@@ -155,7 +171,7 @@ class LayerInputs:
     capacity: int
 
 
-def make_weights(shape: LayerShape, gen: torch.Generator):
+def make_weights(shape: LayerShape, gen: torch.Generator, pow2_scales: bool = False):
     H, I, E = shape.hidden, shape.intermediate, shape.num_weight_experts
     w13 = np.empty((E, 2 * I, H), np.uint8)
     w13s = np.empty((E, 2 * I // QBLOCK, H // QBLOCK), np.float32)
@@ -163,10 +179,10 @@ def make_weights(shape: LayerShape, gen: torch.Generator):
     w2s = np.empty((E, H // QBLOCK, I // QBLOCK), np.float32)
     for e in range(E):
         a = torch.randn(2 * I, H, generator=gen, dtype=torch.float32).mul_(1.0 / math.sqrt(H))
-        c, s = quantise_weight(a)
+        c, s = quantise_weight(a, pow2_scales)
         w13[e], w13s[e] = c.numpy(), s.numpy()
         b = torch.randn(H, I, generator=gen, dtype=torch.float32).mul_(1.0 / math.sqrt(I))
-        c, s = quantise_weight(b)
+        c, s = quantise_weight(b, pow2_scales)
         w2[e], w2s[e] = c.numpy(), s.numpy()
     return w13, w13s, w2, w2s
 
@@ -200,7 +216,7 @@ def make_inputs(wl: Workload, weights=None) -> LayerInputs:
     H = sh.hidden
     gen = torch.Generator().manual_seed(int(np.random.SeedSequence(list(wl.seed)).generate_state(1)[0]))
     if weights is None:
-        weights = make_weights(sh, gen)
+        weights = make_weights(sh, gen, wl.pow2_scales)
     else:
         # keep the activation stream independent of whether weights were drawn
         gen = torch.Generator().manual_seed(
@@ -212,7 +228,7 @@ def make_inputs(wl: Workload, weights=None) -> LayerInputs:
     slabs = []
     for m in range(M):
         x = torch.randn(cap, H, generator=gen, dtype=torch.float32)
-        xc, xs = quantise_activation(x)
+        xc, xs = quantise_activation(x, wl.pow2_scales)
         slabs.append(Slab(xc.numpy(), xs.numpy(), None, None))
     for m in range(M):
         ids, w = sample_routing(wl, rng, cap)
@@ -226,19 +242,21 @@ def make_inputs(wl: Workload, weights=None) -> LayerInputs:
 
 
 def make_custom_inputs(shape: LayerShape, counts: Sequence[int], capacity: int, seed: int,
-                       zipf_s: Optional[float] = None, weights=None) -> LayerInputs:
+                       zipf_s: Optional[float] = None, weights=None,
+                       pow2_scales: bool = False) -> LayerInputs:
     """Inputs for an arbitrary slab split (used for ragged and edge-case tests)."""
-    wl = Workload("custom", shape, int(sum(counts)), len(counts), zipf_s, seed=(99, seed))
+    wl = Workload("custom", shape, int(sum(counts)), len(counts), zipf_s, seed=(99, seed),
+                  pow2_scales=pow2_scales)
     sh = shape
     gen = torch.Generator().manual_seed(seed * 7919 + 17)
     if weights is None:
-        weights = make_weights(sh, gen)
+        weights = make_weights(sh, gen, pow2_scales)
     w13, w13s, w2, w2s = weights
     rng = np.random.default_rng([99, seed])
     slabs = []
     for m, n in enumerate(counts):
         x = torch.randn(capacity, sh.hidden, generator=gen, dtype=torch.float32)
-        xc, xs = quantise_activation(x)
+        xc, xs = quantise_activation(x, pow2_scales)
         ids, w = sample_routing(wl, rng, capacity)
         if n < capacity:
             ids[n:] = rng.integers(-1, sh.num_experts_global, size=(capacity - n, sh.top_k))
