@@ -48,9 +48,12 @@ def swiglu(g: np.ndarray, u: np.ndarray) -> np.ndarray:
 
 
 def pow2_ceil(s: np.ndarray) -> np.ndarray:
-    """Smallest power of two >= s (s > 0, float32), exactly: s = m * 2^e, m in [0.5, 1)."""
+    """Smallest power of two >= s (s > 0, float32), exactly: s = m * 2^e, m in [0.5, 1);
+    at least 2^-126, the smallest normal float32 (an 8-bit exponent factor has no
+    subnormal form)."""
     m, e = np.frexp(np.asarray(s, np.float32))
-    return np.ldexp(np.float32(1.0), np.where(m == 0.5, e - 1, e)).astype(np.float32)
+    p = np.ldexp(np.float32(1.0), np.where(m == 0.5, e - 1, e)).astype(np.float32)
+    return np.maximum(p, np.float32(2.0 ** -126))
 
 
 def requant_rows(h: np.ndarray, pow2: bool = False):

@@ -218,6 +218,12 @@ def test_requant_pow2_worked_example():
     assert q0[0, 0] == 0x7E and s0[0, 0] == np.float32(5.0) / np.float32(448.0)
 
 
+def test_pow2_ceil_edges():
+    s = np.array([1.0, 0.75, 2.0 ** -126, 2.0 ** -130, 3e-39, 448.0], np.float32)
+    want = np.array([1.0, 1.0, 2.0 ** -126, 2.0 ** -126, 2.0 ** -126, 512.0], np.float32)
+    assert np.array_equal(ffn.pow2_ceil(s), want)
+
+
 def test_requant_pow2_properties():
     rng = np.random.default_rng(5)
     h = (rng.standard_normal((64, 512)) * np.exp(rng.uniform(-8, 8, (64, 1)))).astype(np.float32)
