@@ -7,7 +7,8 @@
 // (4 x kind::f8f6f4 MMAs of K=32) into one of two TMEM buffers; the epilogue warps read
 // the partial, multiply it by (row scale x weight-block scale) and accumulate in fp32
 // registers ("software promotion": the scales are arbitrary fp32, so they cannot ride on
-// the hardware's UE8M0 block-scale path).
+// the hardware's UE8M0 block-scale path; gemm_mx.cuh holds the block-scale kernel for
+// inputs whose scales are all powers of two).
 //
 // Tilings (the host launches the kernels of the one set on the plan):
 //   PAIR = 1  one CTA per tile; per K block it loads A 128x128 and B 256x128 (48 KiB).
