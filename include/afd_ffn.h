@@ -236,7 +236,7 @@ AFD_API afd_status_t afd_ffn_get_kernel_times(afd_ffn_plan_t plan, float* ms);
  */
 AFD_API afd_status_t afd_ffn_set_tiling(afd_ffn_plan_t plan, int32_t tiling);
 
-/* Synchronise `stream` and report the tiling (1 or 2) the last layer call used. */
+/* Synchronise `stream` and report the tiling (1 to 5) the last layer call used. */
 AFD_API afd_status_t afd_ffn_get_tiling(afd_ffn_plan_t plan, afd_stream_t stream, int32_t* tiling);
 
 /*
