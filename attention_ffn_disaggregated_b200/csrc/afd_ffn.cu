@@ -16,6 +16,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 #include <new>
 
 #include "afd_ffn.h"
@@ -643,15 +644,29 @@ afd_status_t afd_ffn_set_tiling(afd_ffn_plan_t P, int32_t tiling) {
     const afd_ffn_config_t& c = P->cfg;
     const size_t n_img = static_cast<size_t>(P->G) * (2 * c.intermediate / 128) * (c.hidden / 128);
     if (n_img >= (size_t{1} << 31)) return AFD_ERR_UNSUPPORTED;
+    // the images, then one word the check ORs AFD_STATUS_BAD_SCALE into (the plan's
+    // status word is left alone: the weights are refused here, once, synchronously)
     uint8_t* img = nullptr;
-    if (cudaMalloc(&img, n_img * kSfImage) != cudaSuccess) {
+    const size_t img_bytes = n_img * kSfImage;
+    if (cudaMalloc(&img, img_bytes + 16) != cudaSuccess) {
       cudaGetLastError();
       return AFD_ERR_OUT_OF_MEMORY;
     }
-    mx_weight_sf_kernel<<<P->num_sms * 4, 256>>>(P->w.w13_scale, static_cast<int>(n_img), img, P->status);
-    if (cudaGetLastError() != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
+    int* flag = reinterpret_cast<int*>(img + img_bytes);
+    int bad = 0;
+    if (cudaMemset(flag, 0, sizeof(int)) != cudaSuccess) {
       cudaFree(img);
       return AFD_ERR_CUDA;
+    }
+    mx_weight_sf_kernel<<<P->num_sms * 4, 256>>>(P->w.w13_scale, static_cast<int>(n_img), img, flag);
+    if (cudaGetLastError() != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess ||
+        cudaMemcpy(&bad, flag, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) {
+      cudaFree(img);
+      return AFD_ERR_CUDA;
+    }
+    if (bad & AFD_STATUS_BAD_SCALE) {
+      cudaFree(img);
+      return AFD_ERR_INVALID_ARGUMENT;
     }
     P->mx_sfb = img;
   }
@@ -685,12 +700,15 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 uint8_t* g_noalloc_ptr[kMaxDevices] = {};
+std::mutex g_noalloc_mutex;   // guards g_noalloc_ptr and the set-up calls
 
 // Once per device, with that device current: the array's device address (the host-side
 // name of a __device__ array is only a stand-in) and the routing scatter's shared-memory
-// limit.
+// limit. Host threads making their first call at the same time are serialised here; a
+// failed set-up is retried by the next call.
 afd_status_t noalloc_setup(int dev, uint8_t** out) {
   if (dev < 0 || dev >= kMaxDevices) return AFD_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
   if (!g_noalloc_ptr[dev]) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
@@ -789,6 +807,7 @@ extern "C" afd_status_t afd_ffn_route_noalloc(const afd_ffn_config_t* cfg, const
   rp.row_k = d_row_k;
   rp.row_w = d_row_weight;
   rp.status = d_status;
+  rp.tiling = -1;           // routing only: d_sizes[3] = 0
   // every scratch region is fully written before it is read; only the status starts at 0
   if (cudaMemsetAsync(d_status, 0, sizeof(int32_t), stream) != cudaSuccess) return AFD_ERR_CUDA;
   const size_t scatter_smem = sizeof(int32_t) * (static_cast<size_t>(kRouteWarps) * El1 +

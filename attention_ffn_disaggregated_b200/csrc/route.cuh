@@ -42,7 +42,7 @@ struct RouteParams {
   int32_t* mtile2_off;    // [G+1] 256-row m-tiles (CTA-pair tiling); may be null
   int* scan_ticket;       // zero between calls: route_count runs the scan; null: separate
   int32_t* ready;         // [m-tiles] fused GEMM readiness counters, zeroed by the scan; may be null
-  int tiling;             // as set on the plan: 0 (default, = 1) .. 5
+  int tiling;             // as set on the plan: 0 (default, = 1) .. 5; -1: routing only
   int32_t* tok_mt;        // [Tmax] (slab << 24) | row
   int32_t* tok_need;      // [Tmax] contributions this GPU adds to the token
   int32_t* pos;           // [Tmax*K]
@@ -174,8 +174,9 @@ __device__ void route_scan_body(const RouteParams& p, int T, int* s_warp) {
     if (p.mtile2_off) p.mtile2_off[p.G] = base_tiles2;
     p.info[1] = base_rows;
     p.info[2] = base_tiles;
-    // the tiling this call runs (the host launches only its kernels)
-    p.info[3] = p.tiling == 0 ? 1 : p.tiling;
+    // the tiling this call runs (the host launches only its kernels); 0 for routing
+    // without a layer
+    p.info[3] = p.tiling < 0 ? 0 : (p.tiling == 0 ? 1 : p.tiling);
   }
   if (p.ready)
     for (int i = threadIdx.x; i < base_tiles; i += blockDim.x) p.ready[i] = 0;

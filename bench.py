@@ -185,6 +185,24 @@ def cpu_baseline(inp, n_tokens):
                       f"+ grouped SwiGLU FFN + requant + combine; {dt:.1f} s"}
 
 
+L2_NOTE = ("GPU arm: L2 flushed before every timed layer call (256 MiB write, untimed); "
+           "CPU reference arm: not applicable")
+
+
+def workload_config(wl, inp, rt, world: int) -> dict:
+    """The workload as both arms name it: identical keys and values in the GPU line and
+    the reference (oracle) line. `rt` is the oracle's routing or the layer's (same
+    counts, checked bit for bit by the tests)."""
+    sh = inp.shape
+    counts = np.asarray(rt["counts"] if isinstance(rt, dict) else rt.counts)
+    return {"workload": wl.name, "tokens": int(np.sum(inp.counts)), "slabs": wl.num_slabs,
+            "hidden": sh.hidden, "intermediate": sh.intermediate,
+            "local_experts": sh.num_local_experts, "shared_expert": sh.has_shared_expert,
+            "top_k": sh.top_k, "routed_rows": int(counts.sum()),
+            "active_experts": int(np.count_nonzero(counts)),
+            "parallelism": f"replica x{world}", "l2": L2_NOTE}
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -209,12 +227,7 @@ def run_reference(args):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * tot / len(times), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": wl.name, "tokens": T, "slabs": wl.num_slabs,
-                   "hidden": wl.shape.hidden, "intermediate": wl.shape.intermediate,
-                   "local_experts": wl.shape.num_local_experts,
-                   "shared_expert": wl.shape.has_shared_expert, "top_k": wl.shape.top_k,
-                   "routed_rows": int(rt.num_rows), "active_experts": int(np.sum(rt.counts > 0)),
-                   "parallelism": "replica x1"},
+        "config": workload_config(wl, inp, rt, args.gpus),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": os.cpu_count(), "kind": "oracle",
                          "sample": f"{per_step} tokens per step of the {T}-token workload"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -550,19 +563,14 @@ def main():
             "vs_baseline": None,
             "dtype": "fp8_e4m3",
             "data": "synthetic",
-            "config": {"workload": wl.name, "tokens": T, "slabs": wl.num_slabs, "hidden": H,
-                       "intermediate": I, "local_experts": inp.shape.num_local_experts,
-                       "shared_expert": inp.shape.has_shared_expert, "top_k": inp.shape.top_k,
-                       "routed_rows": R, "active_experts": active,
-                       "gemm_tiling": {1: "one CTA per 128x256 tile, W13 and W2 as two launches",
-                                       4: "one CTA per 128x256 tile, W13 and W2 in one persistent launch",
-                                       2: "CTA pairs on 256x256 tiles (cta_group::2)",
-                                       3: "one CTA per 128x256 tile, W13 rows by tile::gather4",
-                                       5: "one CTA per 128x256 tile, W13 on the block-scale MMA path "
-                                          "(power-of-two scales), W2 as two-launch"}[tiling],
-                       "l2": "flushed between steps (256 MiB write, untimed)",
-                       "launch": "CUDA graph replay" if args.graph else "direct launches",
-                       "parallelism": f"replica x{world}"},
+            "config": workload_config(wl, inp, rt, world),
+            "kernel_config": {"gemm_tiling": {1: "one CTA per 128x256 tile, W13 and W2 as two launches",
+                                              4: "one CTA per 128x256 tile, W13 and W2 in one persistent launch",
+                                              2: "CTA pairs on 256x256 tiles (cta_group::2)",
+                                              3: "one CTA per 128x256 tile, W13 rows by tile::gather4",
+                                              5: "one CTA per 128x256 tile, W13 on the block-scale MMA path "
+                                                 "(power-of-two scales), W2 as two-launch"}[tiling],
+                              "launch": "CUDA graph replay" if args.graph else "direct launches"},
             "roofline": {"bound": "tensor", "kernel": dominant, "achieved": achieved,
                          "peak": fp8_peak, "unit": "TFLOP/s", "frac": achieved / fp8_peak,
                          "traffic": profiled_traffic(dominant, wl.name),

@@ -71,8 +71,8 @@ typedef enum {
 #define AFD_STATUS_BAD_ROUTING 0x1 /* id outside [0, E_g) and != -1, or repeated in a token */
 #define AFD_STATUS_TIMEOUT 0x2     /* a bounded device wait expired; outputs are invalid */
 #define AFD_STATUS_BAD_COUNT 0x4   /* some counts[m] < 0 or > slab_capacity; clamped */
-#define AFD_STATUS_BAD_SCALE 0x8   /* tiling 5: a block scale it read is not a positive normal
-                                      power of two; outputs are invalid */
+#define AFD_STATUS_BAD_SCALE 0x8   /* tiling 5: an activation block scale of this call is not a
+                                      positive normal power of two; outputs are invalid */
 
 /* Limits. */
 #define AFD_MAX_SLABS 128
@@ -145,7 +145,10 @@ typedef struct {
 AFD_API afd_status_t afd_ffn_check_config(const afd_ffn_config_t* cfg);
 
 /*
- * Build a plan for one layer on the current CUDA device: validates cfg and weights,
+ * Build a plan for one layer on the current CUDA device. The FFN GPUs hold expert weights
+ * in block-FP8 and keep pre-allocated receive buffers for the tokens the attention GPUs
+ * publish (FastAFD, "Methodology / System Design", items 1-2); the plan is the FFN side's
+ * per-layer state: validates cfg and weights,
  * checks for an sm_100 device, allocates the workspace (cudaMalloc; freed by
  * afd_ffn_destroy), zeroes the combine accumulators and encodes the TMA descriptors of
  * the weights. The weights are read by every later layer call and must stay valid and
@@ -155,7 +158,12 @@ AFD_API afd_status_t afd_ffn_plan(const afd_ffn_config_t* cfg, const afd_ffn_wei
                           afd_ffn_plan_t* out);
 
 /*
- * Enqueue one layer evaluation on `stream`; never synchronises with the host.
+ * Enqueue one layer evaluation on `stream`; never synchronises with the host. This is the
+ * FFN service's compute step between receiving the activations with their routing and
+ * returning the output (vLLM AFD plugin, "FFN service"), run as the FFN GPU's per-layer
+ * work of pull, block-FP8 grouped GEMMs, activation and push-back (FastAFD, "Methodology /
+ * System Design", item 3): routed rows are grouped by expert, W13 + SwiGLU and W2 run as
+ * grouped GEMMs, and each token's top-K-weighted sum is written as bf16 into its slab row.
  * slabs: host array of num_slabs descriptors (read during the call only; the device
  * buffers they point to must stay valid until the stream reaches the work).
  * d_counts: device int32 [num_slabs]. Returns AFD_ERR_INVALID_ARGUMENT for NULL
@@ -165,7 +173,9 @@ AFD_API afd_status_t afd_ffn_plan(const afd_ffn_config_t* cfg, const afd_ffn_wei
 AFD_API afd_status_t afd_ffn_layer(afd_ffn_plan_t plan, const afd_slab_t* slabs, const int32_t* d_counts,
                            afd_stream_t stream);
 
-/* Free the plan and its workspace. NULL is a no-op. Synchronises the device. */
+/* Free the plan and its workspace (the FFN side's per-layer state built by afd_ffn_plan;
+ * FastAFD, "Methodology / System Design", item 2: the receive buffers are pre-allocated and
+ * live as long as the serving instance). NULL is a no-op. Synchronises the device. */
 AFD_API void afd_ffn_destroy(afd_ffn_plan_t plan);
 
 /* Sizes of a plan. */
@@ -224,12 +234,15 @@ AFD_API afd_status_t afd_ffn_get_kernel_times(afd_ffn_plan_t plan, float* ms);
  * 5: as 1, but W13 runs on the tensor core's block-scale path (kind::mxf8f6f4 with UE8M0
  *    factors): TMEM accumulates a tile's whole K loop and the epilogue runs once per
  *    tile. Only for inputs whose activation and W13 block scales are all positive normal
- *    powers of two (each is then exactly its UE8M0 factor); any other scale sets
- *    AFD_STATUS_BAD_SCALE and afd_ffn_get_status then returns AFD_ERR_INVALID_ARGUMENT.
- *    The first selection on a plan allocates the W13 factor images (E * 2I/128 * H/128 *
- *    512 bytes) and builds them with one kernel launch and a device synchronisation
- *    (AFD_ERR_OUT_OF_MEMORY / AFD_ERR_CUDA on failure; call it on the plan's device).
- *    Each layer call then adds one launch (the activation factor images).
+ *    powers of two (each is then exactly its UE8M0 factor). The first selection on a plan
+ *    allocates the W13 factor images (E * 2I/128 * H/128 * 512 bytes), builds them with
+ *    one kernel launch and a device synchronisation, and checks every W13 scale: if one is
+ *    not a positive normal power of two it frees the images, keeps the previous tiling and
+ *    returns AFD_ERR_INVALID_ARGUMENT (AFD_ERR_OUT_OF_MEMORY / AFD_ERR_CUDA on failure; call
+ *    it on the plan's device). Each layer call then adds one launch (the activation factor
+ *    images), which checks that call's activation scales: any other scale sets
+ *    AFD_STATUS_BAD_SCALE, on every such call, and afd_ffn_get_status then returns
+ *    AFD_ERR_INVALID_ARGUMENT.
  * Results are the same within rounding; tilings 2, 3, 4 and 5 exist for tests and
  * measurements. afd_ffn_kernels_per_layer counts the default tiling's launches (tiling 4
  * makes one fewer, tiling 5 one more). Returns AFD_ERR_INVALID_ARGUMENT outside 0..5.
@@ -268,7 +281,8 @@ AFD_API afd_status_t afd_ffn_inject_stall(afd_ffn_plan_t plan, int32_t enable);
  * cfg, slabs (host array [num_slabs]) and d_counts: as for afd_ffn_plan/afd_ffn_layer
  * (only topk_ids, topk_weights and y of each slab are used; y rows of tokens that receive
  * no contribution are set to zero, as afd_ffn_layer does). Outputs, all caller-owned
- * device memory: d_sizes int32[4] = {T, R, m-tiles, 0}; d_group_count int32[G];
+ * device memory: d_sizes int32[4] = {T, R, m-tiles, 0} (T tokens, R routed rows, the
+ * number of 128-row GEMM tiles over all groups, and 0); d_group_count int32[G];
  * d_group_offset int32[G+1]; d_row_token, d_row_k int32[max_rows] and d_row_weight
  * fp32[max_rows] (max_rows = M*cap*(min(K,E_l)+S)); d_pos int32[M*cap*K];
  * d_status int32[1] (cleared, then OR-ed with AFD_STATUS_* bits).

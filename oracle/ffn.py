@@ -11,9 +11,6 @@ the FFN output, return it). Readings of what the pages leave open:
     scale = amax/448 (scale 1 for an all-zero block) before W2. The quantisation decision
     (the division h/scale and the rounding to e4m3) is taken in float32, the precision the
     GPU kernel takes it in; everything else is float64;
-  * power-of-two mode (pow2_intermediate=True), for layers whose input and weight block
-    scales are all powers of two: the intermediate's block scale is amax/448 rounded up to
-    the next power of two too, so every scale in the layer is an exact UE8M0 factor;
   * combine: out[g] = sum over local slots k (ascending) of w[g,k] * Y[row of (g,k)]
     + S * Y[shared row of g], rounded once to bf16 (RNE); a token with no contribution
     gets exact zeros. topk_weights are used as given (renormalised over all K ids by the
@@ -47,18 +44,8 @@ def swiglu(g: np.ndarray, u: np.ndarray) -> np.ndarray:
     return g * u / (1.0 + np.exp(-g))
 
 
-def pow2_ceil(s: np.ndarray) -> np.ndarray:
-    """Smallest power of two >= s (s > 0, float32), exactly: s = m * 2^e, m in [0.5, 1);
-    at least 2^-126, the smallest normal float32 (an 8-bit exponent factor has no
-    subnormal form)."""
-    m, e = np.frexp(np.asarray(s, np.float32))
-    p = np.ldexp(np.float32(1.0), np.where(m == 0.5, e - 1, e)).astype(np.float32)
-    return np.maximum(p, np.float32(2.0 ** -126))
-
-
-def requant_rows(h: np.ndarray, pow2: bool = False):
-    """Per row, per 128 channels: s = amax/448 (1 if amax == 0), rounded up to a power of
-    two when `pow2`; q = e4m3(h/s).
+def requant_rows(h: np.ndarray):
+    """Per row, per 128 channels: s = amax/448 (1 if amax == 0); q = e4m3(h/s).
 
     Returns (codes uint8 [n, C], scales float32 [n, C/128], dequantised float64 [n, C]).
     The decision is taken in float32.
@@ -68,19 +55,17 @@ def requant_rows(h: np.ndarray, pow2: bool = False):
     hb = h32.reshape(n, C // QB, QB)
     amax = np.abs(hb).max(axis=2) if n else np.zeros((0, C // QB), np.float32)
     s = np.where(amax > 0, amax / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float32)
-    if pow2:
-        s = pow2_ceil(s)
     ratio = (hb / s[:, :, None]).astype(np.float32)
     q = e4m3_encode(ratio)
     hq = e4m3_decode(q) * s[:, :, None].astype(np.float64)
     return q.reshape(n, C), s, hq.reshape(n, C)
 
 
-def expert_forward(x: np.ndarray, w13: np.ndarray, w2: np.ndarray, I: int, pow2: bool = False):
+def expert_forward(x: np.ndarray, w13: np.ndarray, w2: np.ndarray, I: int):
     """One expert on dequantised rows x [r, H] with dequantised W13 [2I, H], W2 [H, I]."""
     G = x @ w13.T
     h = swiglu(G[:, :I], G[:, I:])
-    q, s, hq = requant_rows(h, pow2)
+    q, s, hq = requant_rows(h)
     return hq @ w2.T, q, s
 
 
@@ -103,7 +88,7 @@ def route_inputs(inp) -> Routing:
 
 
 def ffn_layer(inp, tokens: Optional[Sequence[int]] = None, routing: Optional[Routing] = None,
-              keep_intermediates: bool = False, pow2_intermediate: bool = False):
+              keep_intermediates: bool = False):
     """Grouped form: rows grouped by expert, one dense product per expert.
 
     Returns a dict with 'out' (float64 [n, H], before bf16 rounding), 'out_bf16'
@@ -131,7 +116,7 @@ def ffn_layer(inp, tokens: Optional[Sequence[int]] = None, routing: Optional[Rou
         x = dequant_rows(xc[rt.row_token[rows]], xs[rt.row_token[rows]])
         w13 = dequant_weight(inp.w13[e], inp.w13_scale[e])
         w2 = dequant_weight(inp.w2[e], inp.w2_scale[e])
-        y, q, s = expert_forward(x, w13, w2, I, pow2_intermediate)
+        y, q, s = expert_forward(x, w13, w2, I)
         Y[rows] = y
         if keep_intermediates:
             h_codes[rows], h_scales[rows] = q, s
@@ -152,7 +137,7 @@ def ffn_layer(inp, tokens: Optional[Sequence[int]] = None, routing: Optional[Rou
     return res
 
 
-def ffn_layer_bruteforce(inp, pow2_intermediate: bool = False) -> np.ndarray:
+def ffn_layer_bruteforce(inp) -> np.ndarray:
     """Per-token twin: no permutation, one expert evaluation per (token, slot).
 
     Applies the same slot rules independently: -1 skipped; ids outside [0, E_g) or
@@ -178,13 +163,11 @@ def ffn_layer_bruteforce(inp, pow2_intermediate: bool = False) -> np.ndarray:
                     continue
                 e = i - e0
                 y, _, _ = expert_forward(x, dequant_weight(inp.w13[e], inp.w13_scale[e]),
-                                         dequant_weight(inp.w2[e], inp.w2_scale[e]), I,
-                                         pow2_intermediate)
+                                         dequant_weight(inp.w2[e], inp.w2_scale[e]), I)
                 acc += np.float64(sl.topk_weights[t, k]) * y[0]
             if S:
                 y, _, _ = expert_forward(x, dequant_weight(inp.w13[El], inp.w13_scale[El]),
-                                         dequant_weight(inp.w2[El], inp.w2_scale[El]), I,
-                                         pow2_intermediate)
+                                         dequant_weight(inp.w2[El], inp.w2_scale[El]), I)
                 acc += y[0]
             outs.append(acc)
     return np.array(outs).reshape(len(outs), H)

@@ -68,3 +68,42 @@ def compare_outputs(gpu_bits: np.ndarray, oracle_out: np.ndarray, tokens=None, t
     worst = float(ratio.max()) if ratio.size else 0.0
     assert worst <= tol, f"worst row error {worst:.4g} x RMS (tolerance {tol})"
     return worst
+
+
+def structural_tokens(ort, slab_counts, n_total: int, num_routed_groups: int,
+                      seed: int = 0) -> np.ndarray:
+    """Tokens whose rows cover the layer's structure, for workloads too large to check
+    every token against the oracle (all tokens when T <= n_total):
+
+      * the first and last token of every non-empty slab (slab boundaries);
+      * for every group with rows: the tokens of its first row, of the first row of its
+        last 128-row tile and of its last row (ragged last tiles);
+      * every token routed to the coolest active routed expert;
+      * random tokens up to n_total.
+    """
+    T = ort.num_tokens
+    if T <= n_total:
+        return np.arange(T)
+    sel = set()
+    base = np.concatenate([[0], np.cumsum(np.asarray(slab_counts, np.int64))])
+    for m in range(len(slab_counts)):
+        if slab_counts[m] > 0:
+            sel.update((int(base[m]), int(base[m + 1]) - 1))
+    counts, offsets, row_token = ort.counts, ort.offsets, ort.row_token
+    for e in range(counts.size):
+        c = int(counts[e])
+        if c == 0:
+            continue
+        o = int(offsets[e])
+        sel.update(int(row_token[r]) for r in (o, o + ((c - 1) // 128) * 128, o + c - 1))
+    routed = counts[:num_routed_groups]
+    active = np.flatnonzero(routed > 0)
+    if active.size:
+        e = int(active[np.argmin(routed[active])])
+        sel.update(int(t) for t in row_token[offsets[e]:offsets[e + 1]])
+    rng = np.random.default_rng(seed)
+    rest = np.setdiff1d(np.arange(T), np.fromiter(sel, np.int64))
+    need = max(0, n_total - len(sel))
+    if need:
+        sel.update(int(t) for t in rng.choice(rest, size=min(need, rest.size), replace=False))
+    return np.array(sorted(sel), np.int64)

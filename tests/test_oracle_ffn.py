@@ -201,50 +201,13 @@ def test_no_contribution_rows_are_zero():
     assert np.all(out[0] == 0) and np.all(out[1] == 0) and np.any(out[2] != 0)
 
 
-# ------------------------------------------------- power-of-two intermediate scales
+# ------------------------------------------------- power-of-two block scales (inputs)
 
-def test_requant_pow2_worked_example():
-    """One row block by hand. amax 5 gives s = 5/448 = 0.01116 (between 2^-7 and 2^-6);
-    rounded up, s = 2^-6 = 0.015625, so 5 -> 320 = 2^8 * 1.25 (code 0 1111 010 = 0x7A),
-    -1.25 -> -80 = -2^6 * 1.25 (0xEA), 0.3 -> 19.2, nearest e4m3 value 20 = 2^4 * 1.25
-    (0x5A), 0 -> 0. Without the rounding, 5 maps to 448 (0x7E)."""
-    h = np.zeros((1, 128), np.float32)
-    h[0, :3] = [5.0, -1.25, 0.3]
-    q, s, hq = ffn.requant_rows(h, pow2=True)
-    assert s[0, 0] == np.float32(2.0 ** -6)
-    assert list(q[0, :4]) == [0x7A, 0xEA, 0x5A, 0x00]
-    assert hq[0, 0] == 5.0 and hq[0, 1] == -1.25 and hq[0, 2] == 20 * 2.0 ** -6
-    q0, s0, _ = ffn.requant_rows(h)
-    assert q0[0, 0] == 0x7E and s0[0, 0] == np.float32(5.0) / np.float32(448.0)
-
-
-def test_pow2_ceil_edges():
-    s = np.array([1.0, 0.75, 2.0 ** -126, 2.0 ** -130, 3e-39, 448.0], np.float32)
-    want = np.array([1.0, 1.0, 2.0 ** -126, 2.0 ** -126, 2.0 ** -126, 512.0], np.float32)
-    assert np.array_equal(ffn.pow2_ceil(s), want)
-
-
-def test_requant_pow2_properties():
-    rng = np.random.default_rng(5)
-    h = (rng.standard_normal((64, 512)) * np.exp(rng.uniform(-8, 8, (64, 1)))).astype(np.float32)
-    h[3, 128:256] = 0.0                                   # an all-zero block keeps scale 1
-    h[5, :128] = 0.0
-    h[5, 7] = 448.0 * 2.0 ** -5                           # amax/448 already a power of two
-    q, s, hq = ffn.requant_rows(h, pow2=True)
-    q0, s0, _ = ffn.requant_rows(h)
-    bits = s.view(np.uint32)
-    assert np.all((bits & 0x807FFFFF) == 0)               # positive powers of two
-    assert np.all(s >= s0) and np.all(s < 2 * s0)
-    assert s[3, 1] == 1.0
-    assert s[5, 0] == s0[5, 0] and np.array_equal(q[5, :128], q0[5, :128])
-    dec = np.abs(hq / np.repeat(s.astype(np.float64), 128, axis=1))
-    assert np.all(dec <= 448.0)
-
-
-def test_grouped_equals_bruteforce_pow2():
+def test_grouped_equals_bruteforce_pow2_inputs():
+    """The same layer definition on inputs whose block scales are powers of two (the
+    inputs of the block-scale W13 tiling): grouped form and per-token twin agree."""
     inp = W.make_inputs(W.CONFIGS["tiny_pow2"])
-    g = ffn.ffn_layer(inp, pow2_intermediate=True, keep_intermediates=True)
-    b = ffn.ffn_layer_bruteforce(inp, pow2_intermediate=True)
+    g = ffn.ffn_layer(inp, keep_intermediates=True)
+    b = ffn.ffn_layer_bruteforce(inp)
     scale = np.sqrt((b ** 2).mean(axis=1, keepdims=True))
     assert np.max(np.abs(g["out"] - b) / scale) < 1e-9
-    assert np.all((g["h_scales"].view(np.uint32) & 0x807FFFFF) == 0)

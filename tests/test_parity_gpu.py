@@ -11,7 +11,7 @@ import pytest
 
 import workloads as W
 from oracle import ffn as offn
-from tests.helpers import compare_outputs, compare_routing, run_cuda_layer
+from tests.helpers import compare_outputs, compare_routing, run_cuda_layer, structural_tokens
 
 pytestmark = pytest.mark.gpu
 
@@ -92,13 +92,38 @@ def test_block_scale_tiling_limits():
     assert res["tiling"] == 5 and res["status_rc"] == 0
 
 
-def test_block_scale_tiling_flags_other_scales():
-    """amax/448 scales are not powers of two: tiling 5 must flag them (the outputs are then
-    invalid; nothing faults)."""
-    from attention_ffn_disaggregated_b200.ffn import STATUS_BAD_SCALE
+def test_block_scale_tiling_refuses_other_weight_scales():
+    """amax/448 W13 scales are not powers of two: selecting the block-scale tiling is
+    refused synchronously, the plan keeps its tiling and the next call is correct."""
+    from attention_ffn_disaggregated_b200 import AfdError, FfnLayer
+    from attention_ffn_disaggregated_b200.device import to_device_weights
     inp = W.make_inputs(W.CONFIGS["tiny"])
-    res = run_cuda_layer(inp, tiling=5)
-    assert res["status_rc"] == 1 and res["status_word"] & STATUS_BAD_SCALE
+    layer = FfnLayer(inp.shape, len(inp.slabs), inp.capacity, *to_device_weights(inp))
+    with pytest.raises(AfdError) as e:
+        layer.set_tiling(5)
+    assert e.value.code == 1
+    res = run_cuda_layer(inp, layer=layer)
+    assert res["status_rc"] == 0 and res["tiling"] == 1
+    compare_outputs(res["outs"][0], offn.ffn_layer(inp)["out"])
+
+
+def test_block_scale_tiling_flags_activation_scales_on_every_call():
+    """Power-of-two W13 scales but amax/448 activation scales: every tiling-5 call sets
+    BAD_SCALE, also after afd_ffn_get_status has cleared the word."""
+    from attention_ffn_disaggregated_b200 import FfnLayer
+    from attention_ffn_disaggregated_b200.device import (to_device_counts, to_device_slabs,
+                                                          to_device_weights)
+    from attention_ffn_disaggregated_b200.ffn import STATUS_BAD_SCALE
+    sh = W.LayerShape(256, 128, 8, 0, 8, 1, 2)
+    wts = W.make_custom_inputs(sh, [40], 40, seed=41, pow2_scales=True)
+    acts = W.make_custom_inputs(sh, [40], 40, seed=41)
+    layer = FfnLayer(sh, 1, 40, *to_device_weights(wts))
+    layer.set_tiling(5)
+    slabs, counts = to_device_slabs(acts), to_device_counts(acts)
+    for _ in range(2):
+        layer(slabs, counts)
+        rc, word = layer.status()
+        assert rc == 1 and word & STATUS_BAD_SCALE
 
 
 def test_repeated_calls_self_clean():
@@ -190,29 +215,27 @@ def test_timeout_injection_reports_status_and_recovers():
 
 # ------------------------------------------------------------------ full-size workloads
 
-def _sampled_check(name, n_sample=40, tiling=0):
-    wl = W.CONFIGS[name]
-    inp = W.make_inputs(wl)
+def _full_size_check(inp, n_total=None, tiling=0):
+    """Routing bit-exact on every token; outputs against the oracle on every token, or on
+    the structural selection of tests.helpers.structural_tokens when n_total is given."""
     res = run_cuda_layer(inp, tiling=tiling)
-    assert res["status_rc"] == 0
+    assert res["status_rc"] == 0, res["status_word"]
     ort = offn.route_inputs(inp)
     compare_routing(res["routing"], ort)
-    rng = np.random.default_rng(0)
-    T = ort.num_tokens
-    toks = np.unique(np.concatenate([[0, T - 1], rng.choice(T, size=min(n_sample, T), replace=False)]))
+    toks = (None if n_total is None else
+            structural_tokens(ort, inp.counts, n_total, inp.shape.num_local_experts))
     ref = offn.ffn_layer(inp, tokens=toks, routing=ort)
-    return compare_outputs(res["outs"][0], ref["out"], tokens=toks)
+    return compare_outputs(res["outs"][0], ref["out"], tokens=toks), res
 
 
 @pytest.mark.parametrize("name,tiling", [("qwen3_235b_t2048", 0), ("deepseek_v3_share_t4096", 0),
-                                         ("deepseek_v3_share_t4096", 2),
-                                         ("deepseek_v3_share_t4096", 3),
-                                         ("deepseek_v3_share_t4096", 4),
-                                         ("deepseek_v3_share_t4096_pow2", 0),
-                                         ("deepseek_v3_share_t4096_pow2", 5),
-                                         ("qwen3_235b_spec_q4_t8192", 0)])
-def test_full_size_sampled(name, tiling):
-    _sampled_check(name, tiling=tiling)
+                                         ("qwen3_235b_spec_q4_t8192", 0),
+                                         ("deepseek_v3_share_t4096_pow2", 5)])
+def test_full_size_every_token(name, tiling):
+    """The three full-size workloads (and the block-scale tiling on the power-of-two twin of
+    the DeepSeek-V3 share): every output row against the oracle."""
+    _, res = _full_size_check(W.make_inputs(W.CONFIGS[name]), tiling=tiling)
+    assert res["tiling"] == (1 if tiling == 0 else tiling)
 
 
 # --------------------------------------------------------------- sweep cells (T x M)
@@ -224,10 +247,22 @@ def share_weights():
     return W.make_weights(W.DEEPSEEK_V3_SHARE, torch.Generator().manual_seed(4))
 
 
-@pytest.mark.parametrize("cell", ["sweep_t1_m64_uniform", "sweep_t8_m16_zipf1.2", "sweep_t64_m4_uniform"])
-def test_sweep_cells_full_parity(cell, share_weights):
-    """Small-batch cells of the T x M sweep, every output row against the oracle: a single
-    token among 64 slabs (63 empty), a few skewed tokens, and 64 tokens over 4 slabs."""
-    inp = W.make_inputs(W.workload_by_name(cell), weights=share_weights)
-    res, _, _ = _full_check(inp)
-    assert res["status_rc"] == 0
+@pytest.mark.parametrize("cell", ["sweep_t1_m64_uniform", "sweep_t8_m16_zipf1.2", "sweep_t64_m4_uniform",
+                                  "sweep_t512_m1_uniform", "sweep_t512_m64_zipf1.2",
+                                  "sweep_t512_m64_uniform", "sweep_t512_m1_zipf1.2",
+                                  "sweep_t4096_m1_uniform", "sweep_t4096_m64_zipf1.2",
+                                  "sweep_t4096_m64_uniform", "sweep_t4096_m1_zipf1.2"])
+def test_sweep_cells_every_token(cell, share_weights):
+    """Cells of the T x M sweep up to 4096 tokens, every output row against the oracle: a
+    single token among 64 slabs (63 empty), skewed and uniform routing, one slab holding
+    every token and 64 slabs of 8 to 64 tokens."""
+    _full_size_check(W.make_inputs(W.workload_by_name(cell), weights=share_weights))
+
+
+@pytest.mark.parametrize("cell", ["sweep_t16384_m1_uniform", "sweep_t16384_m64_zipf1.2",
+                                  "sweep_t16384_m64_uniform", "sweep_t16384_m1_zipf1.2"])
+def test_sweep_cells_16384_structural(cell, share_weights):
+    """The 16384-token cells (up to ~110k routed rows): routing on every token, outputs on
+    the structural selection (slab ends, every group's first row and both ends of its last
+    tile, all tokens of the coolest expert) topped up to 2048 tokens."""
+    _full_size_check(W.make_inputs(W.workload_by_name(cell), weights=share_weights), n_total=2048)

@@ -45,6 +45,9 @@ def test_noalloc_routing_matches_layer_two_calls(name, make):
         T, R = int(o["sizes"][0]), int(o["sizes"][1])
         K = inp.shape.top_k
         assert T == rt["num_tokens"] and R == rt["num_rows"], call
+        # m-tiles: 128-row GEMM tiles over all groups; the last entry is documented as 0
+        assert int(o["sizes"][2]) == int(np.sum((rt["counts"] + 127) // 128)), call
+        assert int(o["sizes"][3]) == 0, call
         assert np.array_equal(o["counts"], rt["counts"])
         assert np.array_equal(o["offsets"], rt["offsets"])
         assert np.array_equal(o["row_token"][:R], rt["row_token"])
