@@ -26,6 +26,21 @@
 
 using namespace afd;
 
+// Tile order of the down projection: 0 = m-tile major, 1 = column-tile major (every
+// m-tile of a 256-column slice before the next slice).
+#ifndef AFD_W2_SLICE_FIRST
+#define AFD_W2_SLICE_FIRST 0
+#endif
+// With a shared expert the down projection's shared tiles finish the combine (1); 0 keeps
+// the separate finalisation kernel for every layer.
+#ifndef AFD_FUSE_COMBINE
+#define AFD_FUSE_COMBINE 1
+#endif
+
+namespace {
+bool fused_combine(const afd_ffn_config_t& c) { return AFD_FUSE_COMBINE && c.has_shared_expert; }
+}  // namespace
+
 namespace {
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -56,24 +71,23 @@ struct afd_ffn_plan_s {
   int G = 0, Tmax = 0, Rmax = 0, rpad = 0, num_chunks = 0;
   void* ws = nullptr;
   size_t ws_bytes = 0;
-  int32_t *slab_base, *info, *chunk_hist, *chunk_off, *group_count, *group_off, *mtile_off,
-      *mtile2_off;
-  int tiling = 0;  // 0 = chosen per call on the device; 1 / 2 forced
+  int32_t *slab_base, *info, *chunk_hist, *chunk_off, *group_count, *group_off, *mtile_off;
+  int tiling = 0;  // 0 = default (1); 2 = block-scale W13
   int32_t *tok_mt, *tok_need, *pos, *row_token, *row_k;
+  int32_t *blk_need = nullptr, *blk_cnt = nullptr;   // fused combine (shared expert only)
+  float* g_ws;        // split-K W13: fp32 sums [g_rows][2I], zero between calls
+  int g_rows = 0;
+  int* g_cnt;         // split-K W13: per (tile, quadrant) counters [num_sms][4]
   float *row_w, *sa_t, *sh_t, *acc;
   uint8_t *a_perm, *hq;
   int* status;
   int* scan_ticket;   // route_count's last-block counter, zero between calls
-  int32_t* ready;     // fused W13->W2 launch: per m-tile readiness counters
-  // tiling 5 (block-scale W13): factor images of the activation rows (workspace) and of
+  // tiling 2 (block-scale W13): factor images of the activation rows (workspace) and of
   // W13 (allocated and built when the tiling is first selected)
   uint8_t* mx_sfa;
   uint8_t* mx_sfb = nullptr;
   CUtensorMap tm_a13, tm_w13, tm_a2, tm_w2;
-  // tiling 3 (W13 rows gathered from the slabs): one map per slab, re-encoded when a slab's
-  // row pointer changes between calls
-  AMaps<true> slab_maps;
-  const void* slab_x[AFD_MAX_SLABS] = {};
+  int w2_slice_first = AFD_W2_SLICE_FIRST;
   bool timing = false, ev_valid = false;
   cudaEvent_t ev[AFD_NUM_KERNELS + 1] = {};
   unsigned long long wait_limit_ns = 1000000000ull;
@@ -96,8 +110,12 @@ const char* afd_status_string(afd_status_t s) {
   return "unknown";
 }
 
-// default tiling: route count (+ scan), scatter, gather, W13, W2, finalize
-int32_t afd_ffn_kernels_per_layer(void) { return 6; }
+// route count (+ scan), scatter, gather, W13, W2 and, without a shared expert, the
+// finalisation; the block-scale tiling adds the activation factor images
+int32_t afd_ffn_kernels_per_layer(afd_ffn_plan_t P) {
+  if (!P) return -1;
+  return 5 + (fused_combine(P->cfg) ? 0 : 1) + (P->tiling == 2 ? 1 : 0);
+}
 
 afd_status_t afd_ffn_check_config(const afd_ffn_config_t* c) {
   if (!c) return AFD_ERR_INVALID_ARGUMENT;
@@ -138,19 +156,6 @@ static afd_status_t encode_2d(EncodeTiledFn enc, CUtensorMap* m, void* base, uin
   return r == CUDA_SUCCESS ? AFD_OK : AFD_ERR_CUDA;
 }
 
-// A slab's FP8 rows [cap][H] for tile::gather4: box {128 columns, 1 row}.
-static afd_status_t encode_slab(EncodeTiledFn enc, CUtensorMap* m, const void* x, uint64_t H,
-                                uint64_t cap) {
-  cuuint64_t dims[2] = {H, cap};
-  cuuint64_t strides[1] = {H};
-  cuuint32_t box[2] = {128, 1};
-  cuuint32_t es[2] = {1, 1};
-  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(x), dims, strides, box, es,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? AFD_OK : AFD_ERR_CUDA;
-}
-
 static afd_status_t encode_3d(EncodeTiledFn enc, CUtensorMap* m, const void* base, uint64_t inner,
                               uint64_t rows, uint64_t experts, uint32_t box_rows) {
   cuuint64_t dims[3] = {inner, rows, experts};
@@ -185,13 +190,9 @@ afd_status_t afd_ffn_plan(const afd_ffn_config_t* cfg, const afd_ffn_weights_t* 
   // The GEMM kernels split the block's registers between warpgroups with setmaxnreg; that
   // is only safe when the block is launched with exactly the budget the split assumes.
   {
-    const void* fns[7] = {reinterpret_cast<const void*>(grouped_gemm_kernel<EPI_FUSED, 1, false>),
-                          reinterpret_cast<const void*>(w13_mx_kernel),
-                          reinterpret_cast<const void*>(grouped_gemm_kernel<EPI_SWIGLU, 1, false>),
-                          reinterpret_cast<const void*>(grouped_gemm_kernel<EPI_SWIGLU, 1, true>),
-                          reinterpret_cast<const void*>(grouped_gemm_kernel<EPI_SWIGLU, 2, false>),
-                          reinterpret_cast<const void*>(grouped_gemm_kernel<EPI_COMBINE, 1, false>),
-                          reinterpret_cast<const void*>(grouped_gemm_kernel<EPI_COMBINE, 2, false>)};
+    const void* fns[3] = {reinterpret_cast<const void*>(w13_mx_kernel),
+                          reinterpret_cast<const void*>(grouped_gemm_kernel<EPI_SWIGLU>),
+                          reinterpret_cast<const void*>(grouped_gemm_kernel<EPI_COMBINE>)};
     for (const void* fn : fns) {
       cudaFuncAttributes fa;
       if (cudaFuncGetAttributes(&fa, fn) != cudaSuccess) return AFD_ERR_CUDA;
@@ -210,7 +211,8 @@ afd_status_t afd_ffn_plan(const afd_ffn_config_t* cfg, const afd_ffn_weights_t* 
   P->G = El + S;
   P->Tmax = cfg->num_slabs * cfg->slab_capacity;
   P->Rmax = P->Tmax * (std::min(K, El) + S);
-  // a CTA-pair tile may start up to 255 rows before the end of the routed rows
+  // a 128-row tile may start up to 127 rows before the end of the routed rows, and its
+  // row-scale copy reads 132 entries from the 16-byte boundary at or below its first row
   P->rpad = ((P->Rmax + 256 + 127) / 128) * 128;
   P->num_chunks = (P->Tmax + kChunkTokens - 1) / kChunkTokens;
   const int El1 = std::max(El, 1);
@@ -227,15 +229,16 @@ afd_status_t afd_ffn_plan(const afd_ffn_config_t* cfg, const afd_ffn_weights_t* 
   const size_t o_info = take(sizeof(int32_t) * 16, 16);
   const size_t o_status = take(sizeof(int32_t) * 4, 16);
   const size_t o_ticket = take(sizeof(int32_t) * 4, 16);
-  const size_t o_ready = take(sizeof(int32_t) * (P->rpad / 128 + P->G + 1), 16);
   const size_t o_chunk_hist = take(sizeof(int32_t) * P->num_chunks * El1, 16);
   const size_t o_chunk_off = take(sizeof(int32_t) * P->num_chunks * El1, 16);
   const size_t o_group_count = take(sizeof(int32_t) * (P->G + 1), 16);
   const size_t o_group_off = take(sizeof(int32_t) * (P->G + 1), 16);
   const size_t o_mtile_off = take(sizeof(int32_t) * (P->G + 1), 16);
-  const size_t o_mtile2_off = take(sizeof(int32_t) * (P->G + 1), 16);
   const size_t o_tok_mt = take(sizeof(int32_t) * P->Tmax, 16);
   const size_t o_tok_need = take(sizeof(int32_t) * P->Tmax, 16);
+  const size_t n_blk = static_cast<size_t>(2) * P->num_chunks;   // 128-token blocks, rounded up
+  const size_t o_blk_need = take(S ? sizeof(int32_t) * n_blk : 0, 16);
+  const size_t o_blk_cnt = take(S ? sizeof(int32_t) * n_blk * (H / 256) : 0, 16);
   const size_t o_pos = take(sizeof(int32_t) * static_cast<size_t>(P->Tmax) * K, 16);
   const size_t o_row_token = take(sizeof(int32_t) * P->rpad, 16);
   const size_t o_row_k = take(sizeof(int32_t) * P->rpad, 16);
@@ -245,6 +248,11 @@ afd_status_t afd_ffn_plan(const afd_ffn_config_t* cfg, const afd_ffn_weights_t* 
   const size_t o_hq = take(static_cast<size_t>(P->rpad) * I, 1024);
   const size_t o_sh_t = take(sizeof(float) * static_cast<size_t>(I / 128) * P->rpad, 256);
   const size_t o_acc = take(sizeof(float) * static_cast<size_t>(P->Tmax) * H, 256);
+  // split-K W13 runs only while its tiles fill at most half of the grid: m-tiles <=
+  // num_sms / (2 * I/128), so that many 128-row tiles bound the rows it touches
+  P->g_rows = std::min(P->rpad, (P->num_sms / (2 * (I / 128)) + 1) * 128);
+  const size_t o_g_ws = take(sizeof(float) * static_cast<size_t>(P->g_rows) * 2 * I, 256);
+  const size_t o_g_cnt = take(sizeof(int) * static_cast<size_t>(P->num_sms) * 4, 16);
   const size_t o_mx_sfa = take(static_cast<size_t>(P->rpad / 128 + P->G) * (H / 128) * kSfImage, 256);
   P->ws_bytes = take(0, 256);
 
@@ -263,15 +271,17 @@ afd_status_t afd_ffn_plan(const afd_ffn_config_t* cfg, const afd_ffn_weights_t* 
   P->info = reinterpret_cast<int32_t*>(b + o_info);
   P->status = reinterpret_cast<int*>(b + o_status);
   P->scan_ticket = reinterpret_cast<int*>(b + o_ticket);
-  P->ready = reinterpret_cast<int32_t*>(b + o_ready);
   P->chunk_hist = reinterpret_cast<int32_t*>(b + o_chunk_hist);
   P->chunk_off = reinterpret_cast<int32_t*>(b + o_chunk_off);
   P->group_count = reinterpret_cast<int32_t*>(b + o_group_count);
   P->group_off = reinterpret_cast<int32_t*>(b + o_group_off);
   P->mtile_off = reinterpret_cast<int32_t*>(b + o_mtile_off);
-  P->mtile2_off = reinterpret_cast<int32_t*>(b + o_mtile2_off);
   P->tok_mt = reinterpret_cast<int32_t*>(b + o_tok_mt);
   P->tok_need = reinterpret_cast<int32_t*>(b + o_tok_need);
+  if (S) {
+    P->blk_need = reinterpret_cast<int32_t*>(b + o_blk_need);
+    P->blk_cnt = reinterpret_cast<int32_t*>(b + o_blk_cnt);
+  }
   P->pos = reinterpret_cast<int32_t*>(b + o_pos);
   P->row_token = reinterpret_cast<int32_t*>(b + o_row_token);
   P->row_k = reinterpret_cast<int32_t*>(b + o_row_k);
@@ -281,6 +291,8 @@ afd_status_t afd_ffn_plan(const afd_ffn_config_t* cfg, const afd_ffn_weights_t* 
   P->hq = b + o_hq;
   P->sh_t = reinterpret_cast<float*>(b + o_sh_t);
   P->acc = reinterpret_cast<float*>(b + o_acc);
+  P->g_ws = reinterpret_cast<float*>(b + o_g_ws);
+  P->g_cnt = reinterpret_cast<int*>(b + o_g_cnt);
   P->mx_sfa = b + o_mx_sfa;
 
   const int E = P->G;
@@ -295,20 +307,12 @@ afd_status_t afd_ffn_plan(const afd_ffn_config_t* cfg, const afd_ffn_weights_t* 
     return st;
   }
   P->scatter_smem = sizeof(int32_t) * (static_cast<size_t>(kRouteWarps) * El1 + kRouteWarps * 32 * K);
-  if (cudaFuncSetAttribute(grouped_gemm_kernel<EPI_FUSED, 1, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(gemm_smem_bytes(EPI_FUSED))) != cudaSuccess ||
-      cudaFuncSetAttribute(w13_mx_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (cudaFuncSetAttribute(w13_mx_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(mx_smem_bytes())) != cudaSuccess ||
-      cudaFuncSetAttribute(grouped_gemm_kernel<EPI_SWIGLU, 1, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(gemm_smem_bytes(EPI_SWIGLU))) != cudaSuccess ||
-      cudaFuncSetAttribute(grouped_gemm_kernel<EPI_SWIGLU, 1, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(gemm_smem_bytes(EPI_SWIGLU))) != cudaSuccess ||
-      cudaFuncSetAttribute(grouped_gemm_kernel<EPI_SWIGLU, 2, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(gemm_smem_bytes(EPI_SWIGLU))) != cudaSuccess ||
-      cudaFuncSetAttribute(grouped_gemm_kernel<EPI_COMBINE, 1, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(gemm_smem_bytes(EPI_COMBINE))) != cudaSuccess ||
-      cudaFuncSetAttribute(grouped_gemm_kernel<EPI_COMBINE, 2, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(gemm_smem_bytes(EPI_COMBINE))) != cudaSuccess ||
+      cudaFuncSetAttribute(grouped_gemm_kernel<EPI_SWIGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(gemm_smem_bytes<EPI_SWIGLU>())) != cudaSuccess ||
+      cudaFuncSetAttribute(grouped_gemm_kernel<EPI_COMBINE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(gemm_smem_bytes<EPI_COMBINE>())) != cudaSuccess ||
       // the limit is a per-function setting shared by every plan: set the largest any
       // configuration can need, so that a later plan never lowers an earlier plan's limit
       cudaFuncSetAttribute(route_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -353,26 +357,6 @@ afd_status_t afd_ffn_get_info(afd_ffn_plan_t P, afd_ffn_plan_info_t* info) {
   return AFD_OK;
 }
 
-// Launch a CTA-pair kernel: clusters of two consecutive CTAs.
-static cudaError_t launch_pair(void (*kernel)(GemmParams, CUtensorMap, CUtensorMap, YTable, AMaps<false>),
-                               int grid,
-                               size_t smem, cudaStream_t stream, const GemmParams& gp,
-                               const CUtensorMap& ta, const CUtensorMap& tb, const YTable& ytab) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid, 1, 1);
-  cfg.blockDim = dim3(kGemmThreads, 1, 1);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kernel, gp, ta, tb, ytab, AMaps<false>{0});
-}
-
 static void fill_route_params(afd_ffn_plan_t P, const int32_t* d_counts, RouteParams& rp) {
   const afd_ffn_config_t& c = P->cfg;
   rp.counts = d_counts;
@@ -394,12 +378,13 @@ static void fill_route_params(afd_ffn_plan_t P, const int32_t* d_counts, RoutePa
   rp.group_count = P->group_count;
   rp.group_off = P->group_off;
   rp.mtile_off = P->mtile_off;
-  rp.mtile2_off = P->mtile2_off;
   rp.scan_ticket = P->scan_ticket;
-  rp.ready = P->ready;
   rp.tiling = P->tiling;
   rp.tok_mt = P->tok_mt;
   rp.tok_need = P->tok_need;
+  rp.blk_need = fused_combine(c) ? P->blk_need : nullptr;
+  rp.blk_cnt = fused_combine(c) ? P->blk_cnt : nullptr;
+  rp.n_ctiles = c.hidden / 256;
   rp.pos = P->pos;
   rp.row_token = P->row_token;
   rp.row_k = P->row_k;
@@ -415,7 +400,6 @@ static void fill_gemm_params(afd_ffn_plan_t P, int epi, GemmParams& gp) {
   gp.info = P->info;
   gp.group_off = P->group_off;
   gp.mtile_off = P->mtile_off;
-  gp.mtile2_off = P->mtile2_off;
   gp.G = P->G;
   gp.rpad = P->rpad;
   gp.I = c.intermediate;
@@ -423,7 +407,6 @@ static void fill_gemm_params(afd_ffn_plan_t P, int epi, GemmParams& gp) {
   gp.status = P->status;
   gp.wait_limit_ns = P->wait_limit_ns;
   gp.row_token = P->row_token;
-  gp.tok_mt = P->tok_mt;
   if (epi == EPI_SWIGLU) {
     gp.n_tiles = c.intermediate / 128;
     gp.num_kb = c.hidden / 128;
@@ -433,6 +416,10 @@ static void fill_gemm_params(afd_ffn_plan_t P, int epi, GemmParams& gp) {
     gp.hq = P->hq;
     gp.sh_t = P->sh_t;
     gp.inject_stall = P->inject_stall;
+    gp.split_ok = 1;
+    gp.g_ws = P->g_ws;
+    gp.g_rows = P->g_rows;
+    gp.g_cnt = P->g_cnt;
   } else {
     gp.n_tiles = c.hidden / 256;
     gp.num_kb = c.intermediate / 128;
@@ -441,6 +428,12 @@ static void fill_gemm_params(afd_ffn_plan_t P, int epi, GemmParams& gp) {
     gp.ws_rows = c.hidden / 128;
     gp.row_w = P->row_w;
     gp.acc = P->acc;
+    gp.slice_first = P->w2_slice_first;
+    gp.fuse_final = fused_combine(c);
+    gp.split_ok = !fused_combine(c);
+    gp.tok_mt = P->tok_mt;
+    gp.blk_need = P->blk_need;
+    gp.blk_cnt = P->blk_cnt;
   }
 }
 
@@ -471,23 +464,7 @@ afd_status_t afd_ffn_layer(afd_ffn_plan_t P, const afd_slab_t* slabs, const int3
     tab.y[m] = static_cast<__nv_bfloat16*>(s.y);
     ytab.y[m] = static_cast<__nv_bfloat16*>(s.y);
   }
-  // tilings 1 (default), 2 and 4 (W13 and W2 in one persistent launch) read an
-  // expert-ordered copy of the rows made by the gather stage; tiling 3 gathers them from
-  // the slabs inside the W13 kernel (tile::gather4)
-  const int tiling = P->tiling == 0 ? 1 : P->tiling;
-  const bool pair = tiling == 2, slab_gather = tiling == 3, fused = tiling == 4, mx = tiling == 5;
-  if (slab_gather) {
-    EncodeTiledFn enc = get_encode_fn();
-    if (!enc) return AFD_ERR_CUDA;
-    for (int m = 0; m < c.num_slabs; ++m) {
-      if (P->slab_x[m] == slabs[m].x) continue;
-      if (encode_slab(enc, &P->slab_maps.m[m], slabs[m].x, c.hidden, c.slab_capacity) != AFD_OK) {
-        P->slab_x[m] = nullptr;
-        return AFD_ERR_CUDA;
-      }
-      P->slab_x[m] = slabs[m].x;
-    }
-  }
+  const bool mx = P->tiling == 2;
   RouteParams rp;
   fill_route_params(P, d_counts, rp);
   GemmParams g13, g2;
@@ -503,48 +480,27 @@ afd_status_t afd_ffn_layer(afd_ffn_plan_t P, const afd_slab_t* slabs, const int3
   if (tm) cudaEventRecord(P->ev[2], stream);
   route_scatter_kernel<<<P->num_chunks, kRouteThreads, P->scatter_smem, stream>>>(rp, tab);
   if (tm) cudaEventRecord(P->ev[3], stream);
-  if (slab_gather) gather_scales_kernel<<<P->num_sms * 4, kRouteThreads, 0, stream>>>(rp, tab);
-  else gather_rows_kernel<<<P->num_sms * 8, kRouteThreads, 0, stream>>>(rp, tab);
+  gather_rows_kernel<<<P->num_sms * 8, kRouteThreads, 0, stream>>>(rp, tab);
   if (tm) cudaEventRecord(P->ev[4], stream);
-  const int grid1 = P->num_sms, grid2 = P->num_sms & ~1;
-  if (fused) {
-    // one persistent launch: every W13 tile, then every W2 tile (the W2 stage time reads
-    // as zero)
-    FusedArgs fa;
-    fa.p2 = g2;
-    fa.tm_a2 = P->tm_a2;
-    fa.tm_b2 = P->tm_w2;
-    fa.ready = P->ready;
-    grouped_gemm_kernel<EPI_FUSED, 1, false><<<grid1, kGemmThreads, gemm_smem_bytes(EPI_FUSED), stream>>>(
-        g13, P->tm_a13, P->tm_w13, ytab, fa);
-  } else if (mx) {
+  const int grid = P->num_sms;
+  if (mx) {
     // factor images of this call's activation rows, then W13 on the block-scale path (the
     // W13 stage time includes the image kernel)
     mx_act_sf_kernel<<<P->num_sms * 4, 128, 0, stream>>>(P->mtile_off, P->group_off, P->G, P->sa_t,
                                                          P->rpad, c.hidden / 128, P->mx_sfa, P->status);
-    w13_mx_kernel<<<grid1, kGemmThreads, mx_smem_bytes(), stream>>>(g13, P->tm_a13, P->tm_w13,
-                                                                   MxArgs{P->mx_sfa, P->mx_sfb});
-  } else if (slab_gather) {
-    grouped_gemm_kernel<EPI_SWIGLU, 1, true><<<grid1, kGemmThreads, gemm_smem_bytes(EPI_SWIGLU), stream>>>(
-        g13, P->tm_a13, P->tm_w13, ytab, P->slab_maps);
-  } else if (!pair) {
-    grouped_gemm_kernel<EPI_SWIGLU, 1, false><<<grid1, kGemmThreads, gemm_smem_bytes(EPI_SWIGLU), stream>>>(
-        g13, P->tm_a13, P->tm_w13, ytab, AMaps<false>{0});
-  } else if (launch_pair(grouped_gemm_kernel<EPI_SWIGLU, 2, false>, grid2, gemm_smem_bytes(EPI_SWIGLU),
-                         stream, g13, P->tm_a13, P->tm_w13, ytab) != cudaSuccess) {
-    return AFD_ERR_CUDA;
+    w13_mx_kernel<<<grid, kGemmThreads, mx_smem_bytes(), stream>>>(g13, P->tm_a13, P->tm_w13,
+                                                                  MxArgs{P->mx_sfa, P->mx_sfb});
+  } else {
+    grouped_gemm_kernel<EPI_SWIGLU><<<grid, kGemmThreads, gemm_smem_bytes<EPI_SWIGLU>(), stream>>>(
+        g13, P->tm_a13, P->tm_w13, ytab);
   }
   if (tm) cudaEventRecord(P->ev[5], stream);
-  if (!fused && !pair) {
-    grouped_gemm_kernel<EPI_COMBINE, 1, false><<<grid1, kGemmThreads, gemm_smem_bytes(EPI_COMBINE), stream>>>(
-        g2, P->tm_a2, P->tm_w2, ytab, AMaps<false>{0});
-  } else if (pair && launch_pair(grouped_gemm_kernel<EPI_COMBINE, 2, false>, grid2,
-                                 gemm_smem_bytes(EPI_COMBINE), stream, g2, P->tm_a2, P->tm_w2,
-                                 ytab) != cudaSuccess) {
-    return AFD_ERR_CUDA;
-  }
+  grouped_gemm_kernel<EPI_COMBINE><<<grid, kGemmThreads, gemm_smem_bytes<EPI_COMBINE>(), stream>>>(
+      g2, P->tm_a2, P->tm_w2, ytab);
   if (tm) cudaEventRecord(P->ev[6], stream);
-  combine_finalize_kernel<<<P->num_sms * 4, 256, 0, stream>>>(P->info, P->tok_mt, P->acc, c.hidden, ytab);
+  // with a shared expert the down projection's shared tiles write the slab rows themselves
+  if (!fused_combine(c))
+    combine_finalize_kernel<<<P->num_sms * 4, 256, 0, stream>>>(P->info, P->tok_mt, P->acc, c.hidden, ytab);
   if (tm) cudaEventRecord(P->ev[7], stream);
   P->ev_valid = tm;
   if (cudaGetLastError() != cudaSuccess) return AFD_ERR_CUDA;
@@ -636,8 +592,8 @@ afd_status_t afd_ffn_set_wait_limit(afd_ffn_plan_t P, int64_t limit_ns) {
 }
 
 afd_status_t afd_ffn_set_tiling(afd_ffn_plan_t P, int32_t tiling) {
-  if (!P || tiling < 0 || tiling > 5) return AFD_ERR_INVALID_ARGUMENT;
-  if (tiling == 5 && !P->mx_sfb) {
+  if (!P || tiling < 0 || tiling > 2) return AFD_ERR_INVALID_ARGUMENT;
+  if (tiling == 2 && !P->mx_sfb) {
     // the W13 factor images, once per plan (the weights are fixed for its lifetime)
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev != P->device) return AFD_ERR_INVALID_ARGUMENT;
@@ -799,7 +755,6 @@ extern "C" afd_status_t afd_ffn_route_noalloc(const afd_ffn_config_t* cfg, const
   rp.group_count = d_group_count;
   rp.group_off = d_group_offset;
   rp.mtile_off = reinterpret_cast<int32_t*>(scratch + o_mtile);
-  rp.mtile2_off = nullptr;
   rp.tok_mt = reinterpret_cast<int32_t*>(scratch + o_tmt);
   rp.tok_need = reinterpret_cast<int32_t*>(scratch + o_tneed);
   rp.pos = d_pos;

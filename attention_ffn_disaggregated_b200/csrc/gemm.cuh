@@ -10,28 +10,25 @@
 // the hardware's UE8M0 block-scale path; gemm_mx.cuh holds the block-scale kernel for
 // inputs whose scales are all powers of two).
 //
-// Tilings (the host launches the kernels of the one set on the plan):
-//   PAIR = 1  one CTA per tile; per K block it loads A 128x128 and B 256x128 (48 KiB).
-//   PAIR = 2  a CTA pair (cluster of two) shares a 256-row tile of one expert: each CTA
-//             loads its own 128 A rows and half of B (32 KiB per K block), the leader
-//             issues cta_group::2 MMAs (M = 256) and each CTA's TMEM receives its rows.
-//             Less operand traffic per MMA and 6 pipeline stages instead of 4, but each
-//             K block needs a partial-ready / partial-drained handshake between the two
-//             SMs; with only one K block of TMEM slack that latency is exposed, and on
-//             the measured workloads this tiling is about 2x slower. Opt-in only.
-//   GATHER    (W13, PAIR = 1) the A rows come straight from the slabs by tile::gather4.
-//   EPI_FUSED (PAIR = 1) W13 and W2 tiles in one persistent launch (see FusedArgs).
-//
-// Warp roles (384 threads): warp 0 issues TMA loads, warp 1 owns TMEM and (leader) issues
-// MMAs, warps 2..3 idle, warps 4..11 are the epilogue (two per TMEM lane quadrant,
-// splitting the columns).
+// Warp roles (384 threads): warp 0 issues TMA loads, warp 1 owns TMEM and issues MMAs,
+// warps 2..3 idle, warps 4..11 are the epilogue (two per TMEM lane quadrant, splitting
+// the columns).
 //
 // Epilogues:
 //   SWIGLU   (W13) columns are [gate 128 | up 128] of intermediate block nt; h = silu(g)*u
 //            is requantised to e4m3 per (row, 128 channels) and stored with its scale.
-//   COMBINE  (W2)  the row's result times its top-K weight is added (fp32 reductions in
-//            L2) into the token's accumulator; combine_finalize_kernel then writes every
-//            token's sum as bf16 into its slab row and clears the accumulator.
+//   COMBINE  (W2)  the row's result times its top-K weight is added into the token's fp32
+//            accumulator by the bulk-copy engine (cp.reduce.async.bulk ... .add.f32: one
+//            512-byte row segment per operation, staged through shared memory), so the
+//            epilogue warps hand the reductions off and return to the next tile's partial
+//            products. With a shared expert (one row per token, in token order, the last
+//            group) the shared expert's tiles are exactly 128-token blocks and come last in
+//            every CTA's tile order: each routed tile, once its reductions are performed,
+//            adds its rows to a counter per (token block, column tile); the shared tile of
+//            that block waits (bounded) until the counter reaches the block's routed-row
+//            count, adds its own rows to the accumulated sums in registers, writes the bf16
+//            result into the tokens' slab rows and clears the accumulator. Without a shared
+//            expert combine_finalize_kernel does the last step.
 #pragma once
 
 #include "ptx.cuh"
@@ -44,9 +41,10 @@ constexpr int kBK = 128;
 constexpr int kGemmThreads = 384;
 constexpr int kEpiWarps = 8;
 constexpr uint32_t kABytes = kTileM * kBK;   // 16 KiB: 128 rows of one K block
-constexpr int kStgStride = 36;               // floats per staging row (32 + 4 pad)
+constexpr uint32_t kBBytes = kBN * kBK;      // 32 KiB: 256 weight rows of one K block
+constexpr uint32_t kStageBytes = kABytes + kBBytes;
 constexpr uint32_t kTmemCols = 512;          // two 256-column fp32 partial buffers
-constexpr int kMaxStages = 6;
+constexpr int kMaxStages = 4;
 // Register split: the block launches with kLaunchRegs per thread; warpgroup 0 (TMA, MMA,
 // two idle warps) drops to kProducerRegs and the two epilogue warpgroups rise to
 // kEpilogueRegs. 128*40 + 256*232 == 384*168, so the increase never waits for registers
@@ -57,43 +55,35 @@ constexpr int kEpilogueRegs = 232;
 static_assert(128 * kProducerRegs + 256 * kEpilogueRegs <= kGemmThreads * kLaunchRegs,
               "register split exceeds the launch allocation");
 
-// EPI_FUSED: one launch runs every W13 tile (SWIGLU epilogue) and then every W2 tile
-// (COMBINE epilogue), single-CTA tiles; see FusedArgs.
-enum EpiKind { EPI_SWIGLU = 0, EPI_COMBINE = 1, EPI_FUSED = 2 };
+enum EpiKind { EPI_SWIGLU = 0, EPI_COMBINE = 1 };
 
-template <int PAIR>
-struct Tiling {
-  static constexpr int kStages = PAIR == 2 ? 6 : 4;
-  static constexpr uint32_t kBBytes = (kBN / PAIR) * kBK;     // B rows held by this CTA
-  static constexpr uint32_t kStageBytes = kABytes + kBBytes;  // per CTA
-  static constexpr uint32_t kTxBytes = PAIR * kStageBytes;    // landing on the leader's barrier
-  static constexpr int kRows = PAIR * kTileM;                 // rows of one (pair) tile
+// Combine staging: per epilogue warp two buffers of 8 rows x 128 fp32 (+16 bytes of
+// padding per row, so that eight lanes storing one float4 each at the same column hit
+// disjoint banks); a buffer row is the source of one 512-byte bulk reduction.
+constexpr int kStgRows = 8;
+constexpr uint32_t kStgRowBytes = 128 * 4 + 16;
+constexpr uint32_t kStgBufBytes = kStgRows * kStgRowBytes;
+constexpr uint32_t kStgWarpBytes = 2 * kStgBufBytes;
+
+template <int EPI>
+struct GemmCfg {
+  // W13 keeps four operand stages; W2 gives one up for the combine staging
+  static constexpr int kStages = EPI == EPI_SWIGLU ? 4 : 3;
+  static constexpr size_t kStaging = EPI == EPI_SWIGLU ? 0 : static_cast<size_t>(kEpiWarps) * kStgWarpBytes;
 };
 
 struct YTable {
   __nv_bfloat16* y[AFD_MAX_SLABS];
 };
 
-// W13 A operand straight from the slabs: one 2D map per slab over its FP8 rows, box one
-// row high ({128 columns, 1 row}) so that tile::gather4 can fetch four arbitrary rows.
-template <bool GATHER>
-struct AMaps {
-  CUtensorMap m[AFD_MAX_SLABS];
-};
-template <>
-struct AMaps<false> {
-  int unused;
-};
-
-
 struct GemmParams {
   const int32_t* info;        // [0] tokens, [1] rows, [2] m-tiles of this call
   const int32_t* group_off;   // [G+1] first row of each group
   const int32_t* mtile_off;   // [G+1] first 128-row m-tile of each group
-  const int32_t* mtile2_off;  // [G+1] first 256-row m-tile of each group
   int G;
   int n_tiles;                // 256-column tiles per m-tile
   int num_kb;                 // K blocks of 128
+  int slice_first;            // tile order: 0 = m-tile major, 1 = column-tile major
   const float* sa_t;          // A scales, [num_kb][rpad]
   int rpad;
   const float* w_scale;       // [E][ws_rows][num_kb]
@@ -103,71 +93,47 @@ struct GemmParams {
   // SWIGLU epilogue outputs
   uint8_t* hq;                // [rpad][I]
   float* sh_t;                // [I/128][rpad]
-  // W13 from the slabs: row -> token -> (slab << 24) | row in slab
-  const int32_t* tok_mt;
-  // COMBINE epilogue inputs/outputs (row_token also for the slab gather)
+  // COMBINE epilogue inputs/outputs
   const int32_t* row_token;
   const float* row_w;
   float* acc;                 // [Tmax][H] fp32, zero between calls
+  // fused combine (layers with a shared expert): the shared expert's tiles finish each
+  // 128-token block x 256-column tile once its routed rows are in (see the epilogue)
+  int fuse_final;
+  const int32_t* tok_mt;      // [Tmax] (slab << 24) | row in slab
+  const int32_t* blk_need;    // [token blocks] target of each counter
+  int32_t* blk_cnt;           // [token blocks][n_tiles], zeroed by the routing
+  // split-K for launches whose tiles fill less than half of the grid: the K blocks of a
+  // tile are shared out among several CTAs. The down projection's partial sums go to the
+  // combine accumulators like any contribution (only without the fused combine); the gate
+  // / up projection's go to the fp32 workspace g_ws [g_rows][2I], and the CTA whose
+  // partial completes a tile's 32-row quadrant (g_cnt) finishes SwiGLU + requantisation
+  // for those rows from it and clears it.
+  int split_ok;
+  float* g_ws;
+  int g_rows;
+  int* g_cnt;                 // [grid][4], zero between calls
   int* status;
   unsigned long long wait_limit_ns;
   int inject_stall;
 };
 
-// The fused launch's second projection. W2 tile (mt, nt) reads the h rows of m-tile mt,
-// written by the epilogues of the W13 tiles (mt, 0 .. p.n_tiles-1): each of their 8
-// epilogue warps adds 1 to ready[mt] (release) after its stores, and the W2 tile's
-// producer and epilogue wait (bounded, acquire) for 8 * p.n_tiles. Every CTA walks its
-// tiles in increasing order and all W13 tiles precede all W2 tiles, so a W13 tile never
-// waits for anything and every wait ends.
-struct FusedArgs {
-  GemmParams p2;
-  CUtensorMap tm_a2;          // h codes [rpad][I]
-  CUtensorMap tm_b2;          // W2 codes [E][H][I]
-  int32_t* ready;             // [m-tiles], zeroed by the routing scan of each call
-};
+constexpr int kMinSplitKb = 4;    // K blocks per split, at least
+constexpr int kMaxSplits = 8;
 
-template <int EPI, bool GATHER>
-struct ExtraArg {
-  using type = AMaps<GATHER>;
-};
-template <>
-struct ExtraArg<EPI_FUSED, false> {
-  using type = FusedArgs;
-};
+// 16-byte multiple: the combine staging that follows it is the source of bulk copies
+// Row scales of the A operand travel with the operands: for every K block the producer
+// bulk-copies the tile's 128 scales (from the 16-byte boundary at or below the tile's
+// first row: 132 floats) into a ring slot that the epilogue warps release after reading.
+constexpr int kScaleSlots = 8;                 // > stages + the MMA's lead over the epilogue
+constexpr int kScaleRowFloats = 132;
+constexpr uint32_t kScaleRowBytes = kScaleRowFloats * 4;
+static_assert(kScaleRowBytes % 16 == 0, "bulk copy size");
 
-__device__ __forceinline__ const CUtensorMap* slab_map(const AMaps<true>& a, int m) { return &a.m[m]; }
-__device__ __forceinline__ const CUtensorMap* slab_map(const AMaps<false>&, int) { return nullptr; }
-__device__ __forceinline__ const CUtensorMap* slab_map(const FusedArgs&, int) { return nullptr; }
-
-// Parameters and operand maps of a tile: the launch's own, or (fused, W2 tile) the
-// second projection's.
-template <class X>
-__device__ __forceinline__ const GemmParams& tile_params(bool w2, const GemmParams& p, const X&) {
-  return p;
-}
-__device__ __forceinline__ const GemmParams& tile_params(bool w2, const GemmParams& p,
-                                                         const FusedArgs& x) {
-  return w2 ? x.p2 : p;
-}
-template <class X>
-__device__ __forceinline__ void tile_maps(bool, const CUtensorMap* a, const CUtensorMap* b, const X&,
-                                          const CUtensorMap** ma, const CUtensorMap** mb) {
-  *ma = a;
-  *mb = b;
-}
-__device__ __forceinline__ void tile_maps(bool w2, const CUtensorMap* a, const CUtensorMap* b,
-                                          const FusedArgs& x, const CUtensorMap** ma,
-                                          const CUtensorMap** mb) {
-  *ma = w2 ? &x.tm_a2 : a;
-  *mb = w2 ? &x.tm_b2 : b;
-}
-template <class X>
-__device__ __forceinline__ int* ready_of(const X&) { return nullptr; }
-__device__ __forceinline__ int* ready_of(const FusedArgs& x) { return x.ready; }
-
-// 16-byte multiple: the combine staging that follows it is accessed as float4
 struct alignas(16) GemmSmem {
+  float sring[kScaleSlots][kScaleRowFloats];   // first: 16-byte aligned rows
+  uint64_t sfull[kScaleSlots];
+  uint64_t sempty[kScaleSlots];
   uint64_t full[kMaxStages];
   uint64_t empty[kMaxStages];
   uint64_t tfull[2];
@@ -177,17 +143,17 @@ struct alignas(16) GemmSmem {
   int abort_flag;
   float amax[2][2][kTileM];
   int32_t mtile[AFD_MAX_GROUPS + 1];
+  int32_t pend[kEpiWarps][4];   // fused combine: {row0, rows, column tile} of a tile to count
 };
-
-constexpr size_t kGemmSmemTiles = static_cast<size_t>(192) * 1024;   // both tilings
 static_assert(sizeof(GemmSmem) % 16 == 0, "staging after GemmSmem must stay 16-byte aligned");
-static_assert(Tiling<1>::kStages * Tiling<1>::kStageBytes == kGemmSmemTiles, "tiling size");
-static_assert(Tiling<2>::kStages * Tiling<2>::kStageBytes == kGemmSmemTiles, "tiling size");
-constexpr size_t kStgBytes = static_cast<size_t>(kEpiWarps) * 16 * kStgStride * sizeof(float);
 
-__host__ __device__ constexpr size_t gemm_smem_bytes(int epi) {
-  return 1024 + kGemmSmemTiles + sizeof(GemmSmem) + (epi != EPI_SWIGLU ? kStgBytes : 0);
+template <int EPI>
+__host__ __device__ constexpr size_t gemm_smem_bytes() {
+  return 1024 + static_cast<size_t>(GemmCfg<EPI>::kStages) * kStageBytes + sizeof(GemmSmem) +
+         GemmCfg<EPI>::kStaging;
 }
+static_assert(gemm_smem_bytes<EPI_SWIGLU>() <= 232448, "W13 shared memory");
+static_assert(gemm_smem_bytes<EPI_COMBINE>() <= 232448, "W2 shared memory");
 
 // A wait that ignores the abort flag; used only to drain copies/MMAs already in flight.
 __device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
@@ -202,15 +168,23 @@ struct TileCoord {
   int e, row0, rows, nt, mt;
 };
 
-// Tile -> (expert, first row of this CTA's 128 rows, valid rows, column tile).
-// `rows` may be <= 0 for the second CTA of a pair on an expert's last tile.
-template <int PAIR>
-__device__ __forceinline__ TileCoord decode_tile(int tile, int n_tiles, const int32_t* s_mtile,
-                                                 int G, const int32_t* group_off, int rank) {
+// Tile -> (expert, first row, valid rows, column tile). Tiles are numbered m-tile major
+// (all column tiles of m-tile 0, then of m-tile 1, ...) or, with slice_first, column-tile
+// major (every m-tile of column tile 0, then of column tile 1, ...).
+__device__ __forceinline__ TileCoord decode_tile(int tile, int n_tiles, int slice_first,
+                                                 const int32_t* s_mtile, int G,
+                                                 const int32_t* group_off) {
   TileCoord c;
-  const int mt = tile / n_tiles;
+  int mt;
+  if (slice_first) {
+    const int n_mt = s_mtile[G];
+    c.nt = tile / n_mt;
+    mt = tile - c.nt * n_mt;
+  } else {
+    mt = tile / n_tiles;
+    c.nt = tile - mt * n_tiles;
+  }
   c.mt = mt;
-  c.nt = tile - mt * n_tiles;
   int lo = 0, hi = G - 1;               // last group whose first m-tile is <= mt
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
@@ -218,42 +192,88 @@ __device__ __forceinline__ TileCoord decode_tile(int tile, int n_tiles, const in
   }
   c.e = lo;
   const int g0 = group_off[lo], g1 = group_off[lo + 1];
-  c.row0 = g0 + (mt - s_mtile[lo]) * Tiling<PAIR>::kRows + rank * kTileM;
+  c.row0 = g0 + (mt - s_mtile[lo]) * kTileM;
   c.rows = min(kTileM, g1 - c.row0);
   return c;
 }
 
-// GATHER (W13, single-CTA tiles only): the A tile's rows are fetched from the slabs
-// through `extra` (AMaps<true>) instead of from the expert-ordered copy behind `tm_a`.
-// EPI_FUSED: `p`, `tm_a`, `tm_b` describe W13 and `extra` (FusedArgs) W2.
-template <int EPI, int PAIR, bool GATHER>
+// silu(g) * u = g / (1 + exp(-g)) * u with branch-free fast exp and division; g is clamped
+// at -80, where silu is 0 to fp32 precision, so exp(-g) stays finite
+__device__ __forceinline__ float silu_mul(float g, float u) {
+  const float gx = fmaxf(g, -80.0f);
+  return __fdividef(gx, 1.0f + __expf(-gx)) * u;
+}
+
+// Split-K W13: one row's SwiGLU + requantisation for intermediate block nt from the fp32
+// sums in G (gate at columns nt*128.., up at I + nt*128..), which are then cleared. The same
+// arithmetic as the one-CTA epilogue, with the row's 128 channels in one thread.
+__device__ __forceinline__ void split_swiglu_row(const GemmParams& p, int row, int nt) {
+  float* gr = p.g_ws + static_cast<size_t>(row) * (2 * p.I) + nt * 128;
+  // two passes over the row's sums in L2: the block amax, then the codes
+  float amax = 0.f;
+#pragma unroll 4
+  for (int i = 0; i < 32; ++i) {
+    const float4 g = __ldcg(reinterpret_cast<const float4*>(gr + 4 * i));
+    const float4 u = __ldcg(reinterpret_cast<const float4*>(gr + p.I + 4 * i));
+    amax = fmaxf(amax, fmaxf(fmaxf(fabsf(silu_mul(g.x, u.x)), fabsf(silu_mul(g.y, u.y))),
+                             fmaxf(fabsf(silu_mul(g.z, u.z)), fabsf(silu_mul(g.w, u.w)))));
+  }
+  const float sc = amax > 0.f ? amax / 448.0f : 1.0f;
+  const float rsc = __frcp_rn(sc);
+  uint32_t* dst = reinterpret_cast<uint32_t*>(p.hq + static_cast<size_t>(row) * p.I + nt * 128);
+#pragma unroll 4
+  for (int i = 0; i < 32; ++i) {
+    const float4 g = __ldcg(reinterpret_cast<const float4*>(gr + 4 * i));
+    const float4 u = __ldcg(reinterpret_cast<const float4*>(gr + p.I + 4 * i));
+    dst[i] = static_cast<uint32_t>(pack_e4m3x2(silu_mul(g.x, u.x) * rsc, silu_mul(g.y, u.y) * rsc)) |
+             (static_cast<uint32_t>(pack_e4m3x2(silu_mul(g.z, u.z) * rsc, silu_mul(g.w, u.w) * rsc)) << 16);
+    __stcg(reinterpret_cast<float4*>(gr + 4 * i), make_float4(0.f, 0.f, 0.f, 0.f));
+    __stcg(reinterpret_cast<float4*>(gr + p.I + 4 * i), make_float4(0.f, 0.f, 0.f, 0.f));
+  }
+  p.sh_t[static_cast<size_t>(nt) * p.rpad + row] = sc;
+}
+
+// Fused combine: this thread's bulk reductions of a routed tile are performed; add its row
+// to the counter of (its token's 128-token block, the tile's column tile), with release
+// semantics, so that the shared tile that reads the block's sums sees them.
+// `pend` is the warp's {row0, rows, column tile} record in shared memory, cleared here.
+// The warp's rows are in token order, so they fall into one or a few token blocks: one
+// release-add per block, by the first lane of its run, after every lane has fenced its own
+// reductions (the warp barrier orders them before that add).
+__device__ __forceinline__ void combine_count(const GemmParams& p, int32_t* pend, int trow, int lane) {
+  const int row0 = pend[0], rows = pend[1], nt = pend[2];
+  bulk_wait_all();
+  fence_proxy_async_global();
+  __threadfence();
+  const int tb = trow < rows ? (p.row_token[row0 + trow] >> 7) : -1;
+  const unsigned same = __match_any_sync(0xffffffffu, tb);
+  __syncwarp();
+  if (tb >= 0 && lane == __ffs(same) - 1)
+    red_release_add(p.blk_cnt + static_cast<size_t>(tb) * p.n_tiles + nt, __popc(same));
+  __syncwarp();
+  if (lane == 0) pend[1] = 0;
+  __syncwarp();
+}
+
+template <int EPI>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ GemmParams p,
                         const __grid_constant__ CUtensorMap tm_a,
                         const __grid_constant__ CUtensorMap tm_b,
-                        const __grid_constant__ YTable ytab,
-                        const __grid_constant__ typename ExtraArg<EPI, GATHER>::type extra) {
-  static_assert(!GATHER || (EPI == EPI_SWIGLU && PAIR == 1), "slab gather: W13, single-CTA tiles");
-  static_assert(EPI != EPI_FUSED || (PAIR == 1 && !GATHER), "fused launch: single-CTA tiles");
-  constexpr bool kFused = EPI == EPI_FUSED;
-  using TL = Tiling<PAIR>;
-  constexpr int kStages = TL::kStages;
+                        const __grid_constant__ YTable ytab) {
+  constexpr int kStages = GemmCfg<EPI>::kStages;
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
   uint8_t* sA = base;
   uint8_t* sB = base + kStages * kABytes;
-  GemmSmem& S = *reinterpret_cast<GemmSmem*>(base + kGemmSmemTiles);
-  float* stg = reinterpret_cast<float*>(base + kGemmSmemTiles + sizeof(GemmSmem));
+  GemmSmem& S = *reinterpret_cast<GemmSmem*>(base + kStages * kStageBytes);
+  uint8_t* stg = base + kStages * kStageBytes + sizeof(GemmSmem);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   volatile int* abort_flag = &S.abort_flag;
-  const uint32_t rank = PAIR == 2 ? cluster_ctarank() : 0;
-  const bool leader = rank == 0;
-  const int unit = PAIR == 2 ? blockIdx.x / 2 : blockIdx.x;    // pair (or CTA) index
-  const int nunits = PAIR == 2 ? gridDim.x / 2 : gridDim.x;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -262,144 +282,63 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&S.tfull[b], 1);
-      mbar_init(&S.tempty[b], kEpiWarps * PAIR);
+      mbar_init(&S.tempty[b], kEpiWarps);
     }
     for (int i = 0; i < 4; ++i) mbar_init(&S.pair[i], 64);
+    for (int i = 0; i < kScaleSlots; ++i) {
+      mbar_init(&S.sfull[i], 1);
+      mbar_init(&S.sempty[i], kEpiWarps);
+    }
     S.abort_flag = 0;
     fence_mbar_init();
   }
-  const int32_t* mtile_src = PAIR == 2 ? p.mtile2_off : p.mtile_off;
-  for (int i = threadIdx.x; i <= p.G; i += blockDim.x) S.mtile[i] = mtile_src[i];
+  for (int i = threadIdx.x; i <= p.G; i += blockDim.x) S.mtile[i] = p.mtile_off[i];
   if (warp == 1) {
-    if (PAIR == 2) {
-      tmem_alloc_pair(&S.tmem_base, kTmemCols);
-      tmem_relinquish_pair();
-    } else {
-      tmem_alloc(&S.tmem_base, kTmemCols);
-      tmem_relinquish();
-    }
+    tmem_alloc(&S.tmem_base, kTmemCols);
+    tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
-  if (PAIR == 2) cluster_sync();     // both CTAs' barriers exist before any remote signal
   tc_fence_after();
   const uint32_t tmem_base = S.tmem_base;
-  // tile sequence: the launch's own tiles [0, T1) and, fused, the W2 tiles after them
-  const int T1 = S.mtile[p.G] * p.n_tiles;
-  int total_tiles = T1;
-  if constexpr (kFused) total_tiles += S.mtile[p.G] * extra.p2.n_tiles;
-  int* ready = ready_of(extra);
-  const int ready_target = kEpiWarps * p.n_tiles;
+  const int nkb = p.num_kb;
+  // split-K when the tiles fill less than half of the grid (small batches)
+  const int n_tiles0 = S.mtile[p.G] * p.n_tiles;
+  int splits = 1;
+  if (p.split_ok && n_tiles0 > 0 && 2 * n_tiles0 <= static_cast<int>(gridDim.x) &&
+      (EPI == EPI_COMBINE || S.mtile[p.G] * kTileM <= p.g_rows))
+    splits = max(1, min(min(static_cast<int>(gridDim.x) / n_tiles0, nkb / kMinSplitKb), kMaxSplits));
+  const int total_units = n_tiles0 * splits;
 
   if (warp < 4) {
     // each role's code sits inside the branch that sets its register budget
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kProducerRegs));
-    if (GATHER && warp == 0) {
-      // ------------------------------------------------- TMA producer, A rows from the slabs
-      // lane l fetches tile rows 4l..4l+3: one gather4 when the four share a slab, else one
-      // single-row copy each; rows past the group's end repeat the tile's first row
-      if (lane == 0) tma_prefetch_desc(&tm_b);
-      const uint64_t pol_a = policy_evict_last();
-      const uint64_t pol_b = policy_evict_last();
-      int it = 0;
-      bool ok = true;
-      int skipped = -1;
-      for (int tile = unit; ok && tile < total_tiles; tile += nunits) {
-        const TileCoord c = decode_tile<PAIR>(tile, p.n_tiles, S.mtile, p.G, p.group_off, rank);
-        const int brow0 = c.nt * 128;            // gate block
-        const int brow1 = p.I + c.nt * 128;      // up block
-        int rm[4], rt[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int r = 4 * lane + j;
-          const int mt = p.tok_mt[p.row_token[c.row0 + (r < c.rows ? r : 0)]];
-          rm[j] = mt >> 24;
-          rt[j] = mt & 0xFFFFFF;
-        }
-        const bool one_slab = rm[0] == rm[1] && rm[0] == rm[2] && rm[0] == rm[3];
-        for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
-          const int s = it % kStages;
-          const uint32_t ph = (it / kStages) & 1;
-          int got = 1;
-          if (lane == 0) got = mbar_wait(&S.empty[s], ph ^ 1, abort_flag, p.status, p.wait_limit_ns);
-          got = __shfl_sync(0xffffffffu, got, 0);
-          if (!got) {
-            ok = false;
-            break;
-          }
-          if (p.inject_stall && blockIdx.x == 0 && it == 0) {
-            skipped = it;       // test hook: never fill this stage
-            continue;
-          }
-          uint8_t* a = sA + s * kABytes + 4 * lane * kBK;
-          uint8_t* b = sB + s * TL::kBBytes;
-          if (lane == 0) {
-            mbar_arrive_expect_tx(&S.full[s], TL::kTxBytes);
-            tma_load_3d(b, &tm_b, &S.full[s], kb * kBK, brow0, c.e, pol_b);
-            tma_load_3d(b + TL::kBBytes / 2, &tm_b, &S.full[s], kb * kBK, brow1, c.e, pol_b);
-          }
-          __syncwarp();
-          if (one_slab) {
-            tma_gather4(a, slab_map(extra, rm[0]), &S.full[s], kb * kBK, rt[0], rt[1], rt[2], rt[3],
-                        pol_a);
-          } else {
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-              tma_load_2d(a + j * kBK, slab_map(extra, rm[j]), &S.full[s], kb * kBK, rt[j], pol_a);
-          }
-        }
-      }
-      if (!ok && lane == 0) {
-        // wait (bounded) for copies that may still be landing on this CTA's barriers
-        for (int j = max(0, it - kStages); j < it; ++j) {
-          if (j == skipped) continue;
-          mbar_wait_drain(&S.full[j % kStages], (j / kStages) & 1, p.wait_limit_ns);
-        }
-      }
-    } else if (!GATHER && warp == 0 && lane == 0) {
+    if (warp == 0 && lane == 0) {
       // ---------------------------------------------------------------- TMA producer
       tma_prefetch_desc(&tm_a);
       tma_prefetch_desc(&tm_b);
-      // A rows are re-read by every column tile of their m-tile; in the down projection
-      // the weights stream past the L2-resident combine accumulators, so they go first.
-      // In the fused launch the W13 operands go first too: within one launch their
-      // evict-last marks would outlive the W13 phase and crowd the W2 phase's L2 working set
-      // (measured: 1582 against 1653 us on the 4096-token DeepSeek-V3 share).
+      // A rows are re-read by every column tile of their m-tile. W13 weight blocks are
+      // re-read by every m-tile of their expert; W2's stream past the L2-resident combine
+      // accumulators, so they go first.
       const uint64_t pol_a = policy_evict_last();
-      const uint64_t pol_a13 = kFused ? policy_evict_first() : pol_a;
+      const uint64_t pol_b = EPI == EPI_SWIGLU ? policy_evict_last() : policy_evict_first();
       int it = 0;
       bool ok = true;
       int skipped = -1;
-      for (int tile = unit; ok && tile < total_tiles; tile += nunits) {
-        const bool w2 = kFused && tile >= T1;
-        const GemmParams& tp = tile_params(w2, p, extra);
-        const CUtensorMap *ma, *mb;
-        tile_maps(w2, &tm_a, &tm_b, extra, &ma, &mb);
-        const TileCoord c = decode_tile<PAIR>(w2 ? tile - T1 : tile, tp.n_tiles, S.mtile, p.G,
-                                              p.group_off, rank);
-        const bool swiglu = EPI == EPI_SWIGLU || (kFused && !w2);
-        // B rows of this tile: [brow0, +128) and [brow1, +128); a pair splits them
+      for (int u = blockIdx.x; ok && u < total_units; u += gridDim.x) {
+        const int tile = u / splits, sp = u - tile * splits;
+        const int kb0 = sp * nkb / splits, kb1 = (sp + 1) * nkb / splits;
+        const TileCoord c = decode_tile(tile, p.n_tiles, p.slice_first, S.mtile, p.G, p.group_off);
+        // B rows of this tile: [brow0, +128) and [brow1, +128)
         int brow0, brow1;
-        if (swiglu) {
+        if (EPI == EPI_SWIGLU) {
           brow0 = c.nt * 128;               // gate block
-          brow1 = tp.I + c.nt * 128;         // up block
+          brow1 = p.I + c.nt * 128;         // up block
         } else {
           brow0 = c.nt * kBN;
           brow1 = c.nt * kBN + 128;
         }
-        const uint64_t pol_b = (swiglu && !kFused) ? policy_evict_last() : policy_evict_first();
-        // loop bounds in registers: the asm memory clobbers of the waits below would
-        // otherwise force reloads through the (run-time selected) parameter reference
-        const int nkb = kFused ? tp.num_kb : p.num_kb;
-        if (w2) {
-          // the h rows of this m-tile are complete once all its W13 tiles have stored them
-          if (!wait_count(ready + c.mt, ready_target, abort_flag, p.status, p.wait_limit_ns)) {
-            ok = false;
-            break;
-          }
-          fence_proxy_async_global();
-        }
-        for (int kb = 0; kb < (kFused ? nkb : p.num_kb); ++kb, ++it) {
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
           const int s = it % kStages;
           const uint32_t ph = (it / kStages) & 1;
           if (!mbar_wait(&S.empty[s], ph ^ 1, abort_flag, p.status, p.wait_limit_ns)) {
@@ -410,78 +349,69 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             skipped = it;       // test hook: never fill this stage
             continue;
           }
-          uint8_t* a = sA + s * kABytes;
-          uint8_t* b = sB + s * TL::kBBytes;
-          if (PAIR == 1) {
-            mbar_arrive_expect_tx(&S.full[s], TL::kTxBytes);
-            tma_load_2d(a, ma, &S.full[s], kb * kBK, c.row0, w2 ? pol_a : pol_a13);
-            tma_load_3d(b, mb, &S.full[s], kb * kBK, brow0, c.e, pol_b);
-            tma_load_3d(b + TL::kBBytes / 2, mb, &S.full[s], kb * kBK, brow1, c.e, pol_b);
-          } else {
-            const uint32_t fb = mapa_shared(smem_u32(&S.full[s]), 0);
-            if (leader) mbar_arrive_expect_tx(&S.full[s], TL::kTxBytes);
-            tma_load_2d_pair(a, &tm_a, fb, kb * kBK, c.row0, pol_a);
-            tma_load_3d_pair(b, &tm_b, fb, kb * kBK, leader ? brow0 : brow1, c.e, pol_b);
+          // the A rows' scales of this K block into the next ring slot
+          const int ss = it % kScaleSlots;
+          if (!mbar_wait(&S.sempty[ss], ((it / kScaleSlots) & 1) ^ 1, abort_flag, p.status, p.wait_limit_ns)) {
+            ok = false;
+            break;
           }
+          mbar_arrive_expect_tx(&S.sfull[ss], kScaleRowBytes);
+          bulk_load(S.sring[ss], p.sa_t + static_cast<size_t>(kb) * p.rpad + (c.row0 & ~3), kScaleRowBytes,
+                    &S.sfull[ss]);
+          uint8_t* a = sA + s * kABytes;
+          uint8_t* b = sB + s * kBBytes;
+          mbar_arrive_expect_tx(&S.full[s], kStageBytes);
+          tma_load_2d(a, &tm_a, &S.full[s], kb * kBK, c.row0, pol_a);
+          tma_load_3d(b, &tm_b, &S.full[s], kb * kBK, brow0, c.e, pol_b);
+          tma_load_3d(b + kBBytes / 2, &tm_b, &S.full[s], kb * kBK, brow1, c.e, pol_b);
         }
       }
-      if (!ok && leader) {
-        // wait (bounded) for copies that may still be landing on this CTA's barriers
+      if (!ok) {
+        // wait (bounded) for copies that may still be landing on this CTA's barriers (a
+        // K block whose stage wait failed issued nothing; its scale copy may have landed)
         for (int j = max(0, it - kStages); j < it; ++j) {
           if (j == skipped) continue;
           mbar_wait_drain(&S.full[j % kStages], (j / kStages) & 1, p.wait_limit_ns);
         }
+        for (int j = max(0, it - kScaleSlots); j < it; ++j) {
+          if (j == skipped) continue;
+          mbar_wait_drain(&S.sfull[j % kScaleSlots], (j / kScaleSlots) & 1, p.wait_limit_ns);
+        }
       }
-    } else if (warp == 1 && lane == 0 && leader) {
+    } else if (warp == 1 && lane == 0) {
       // ---------------------------------------------------------------- MMA issuer
-      constexpr uint32_t idesc = idesc_e4m3_f32(TL::kRows, kBN);
-      int it = 0, kbg = 0;
+      constexpr uint32_t idesc = idesc_e4m3_f32(kTileM, kBN);
+      int it = 0;
       bool ok = true;
-      for (int tile = unit; ok && tile < total_tiles; tile += nunits) {
-        const int num_kb = tile_params(kFused && tile >= T1, p, extra).num_kb;
-        for (int kb = 0; kb < num_kb; ++kb, ++it, ++kbg) {
+      for (int u = blockIdx.x; ok && u < total_units; u += gridDim.x) {
+        const int sp = u % splits;
+        const int nk = (sp + 1) * nkb / splits - sp * nkb / splits;
+        for (int k = 0; k < nk; ++k, ++it) {
           const int s = it % kStages;
           const uint32_t ph = (it / kStages) & 1;
           if (!mbar_wait(&S.full[s], ph, abort_flag, p.status, p.wait_limit_ns)) {
             ok = false;
             break;
           }
-          const int b = kbg & 1;
-          const uint32_t tph = (kbg >> 1) & 1;
-          const bool got = PAIR == 2
-                               ? mbar_wait_cluster(&S.tempty[b], tph ^ 1, abort_flag, p.status,
-                                                   p.wait_limit_ns)
-                               : mbar_wait(&S.tempty[b], tph ^ 1, abort_flag, p.status,
-                                           p.wait_limit_ns);
-          if (!got) {
+          const int b = it & 1;
+          const uint32_t tph = (it >> 1) & 1;
+          if (!mbar_wait(&S.tempty[b], tph ^ 1, abort_flag, p.status, p.wait_limit_ns)) {
             ok = false;
             break;
           }
           tc_fence_after();
           const uint32_t d = tmem_base + b * kBN;
           const uint64_t a0 = sdesc_k_sw128(smem_u32(sA + s * kABytes));
-          const uint64_t b0 = sdesc_k_sw128(smem_u32(sB + s * TL::kBBytes));
-          if (PAIR == 1) {
+          const uint64_t b0 = sdesc_k_sw128(smem_u32(sB + s * kBBytes));
 #pragma unroll
-            for (int k = 0; k < kBK / 32; ++k)
-              umma_e4m3(d, a0 + 2 * k, b0 + 2 * k, idesc, k > 0 ? 1u : 0u);
-            umma_commit(&S.empty[s]);
-            umma_commit(&S.tfull[b]);
-          } else {
-#pragma unroll
-            for (int k = 0; k < kBK / 32; ++k)
-              umma_e4m3_pair(d, a0 + 2 * k, b0 + 2 * k, idesc, k > 0 ? 1u : 0u);
-            // the same barriers in both CTAs: this CTA's and the peer's copy
-            const uint32_t e_own = smem_u32(&S.empty[s]), t_own = smem_u32(&S.tfull[b]);
-            umma_commit_pair(e_own);
-            umma_commit_pair(mapa_shared(e_own, 1));
-            umma_commit_pair(t_own);
-            umma_commit_pair(mapa_shared(t_own, 1));
-          }
+          for (int k32 = 0; k32 < kBK / 32; ++k32)
+            umma_e4m3(d, a0 + 2 * k32, b0 + 2 * k32, idesc, k32 > 0 ? 1u : 0u);
+          umma_commit(&S.empty[s]);
+          umma_commit(&S.tfull[b]);
         }
       }
-      if (!ok && kbg > 0) {
-        const int last = kbg - 1;
+      if (!ok && it > 0) {
+        const int last = it - 1;
         mbar_wait_drain(&S.tfull[last & 1], (last >> 1) & 1, p.wait_limit_ns);
       }
     }
@@ -493,37 +423,25 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int q = warp & 3;                 // TMEM lane quadrant this warp may access
     const int trow = 32 * q + lane;
     const uint32_t tq = tmem_base + (static_cast<uint32_t>(32 * q) << 16);
-    // the MMA issuer waits on the leader's tempty barriers
-    const uint32_t tempty0 = PAIR == 2 ? mapa_shared(smem_u32(&S.tempty[0]), 0) : 0u;
-    const uint32_t tempty1 = PAIR == 2 ? mapa_shared(smem_u32(&S.tempty[1]), 0) : 0u;
     int kbg = 0, titer = 0;
     bool ok = true;
     const uint64_t pol_acc = policy_evict_last();
-    for (int tile = unit; ok && tile < total_tiles; tile += nunits, ++titer) {
-      const bool w2 = kFused && tile >= T1;
-      const GemmParams& tp = tile_params(w2, p, extra);
-      const TileCoord c = decode_tile<PAIR>(w2 ? tile - T1 : tile, tp.n_tiles, S.mtile, p.G,
-                                            p.group_off, rank);
-      const bool swiglu = EPI == EPI_SWIGLU || (kFused && !w2);
+    // fused combine: the last routed tile whose rows are still to be counted (its row0,
+    // rows and column tile in S.pend[ew]; rows == 0: none)
+    int32_t* pend = S.pend[ew];
+    if (lane == 0) pend[1] = 0;
+    __syncwarp();
+    for (int u = blockIdx.x; ok && u < total_units; u += gridDim.x, ++titer) {
+      const int tile = u / splits, sp = u - tile * splits;
+      const int kb0 = sp * nkb / splits, kb1 = (sp + 1) * nkb / splits;
+      const TileCoord c = decode_tile(tile, p.n_tiles, p.slice_first, S.mtile, p.G, p.group_off);
       const int grow = c.row0 + trow;
       const bool valid = trow < c.rows;
-      if (w2) {
-        // the h scales of this m-tile come from other CTAs' W13 epilogues
-        int got = 1;
-        if (lane == 0) got = wait_count(ready + c.mt, ready_target, abort_flag, p.status, p.wait_limit_ns);
-        got = __shfl_sync(0xffffffffu, got, 0);
-        if (!got) {
-          ok = false;
-          break;
-        }
-        ld_acquire(ready + c.mt);
-      }
-      const int nkb = kFused ? tp.num_kb : p.num_kb;
-      const float* wsb = tp.w_scale + static_cast<size_t>(c.e) * tp.ws_rows * nkb;
+      const float* wsb = p.w_scale + static_cast<size_t>(c.e) * p.ws_rows * nkb;
       int rs0, rs1, c0, c1;
-      if (swiglu) {
+      if (EPI == EPI_SWIGLU) {
         rs0 = c.nt;
-        rs1 = tp.I / 128 + c.nt;
+        rs1 = p.I / 128 + c.nt;
         c0 = 64 * half;
         c1 = 128 + 64 * half;
       } else {
@@ -538,17 +456,38 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       float2 acc[64];
 #pragma unroll
       for (int i = 0; i < 64; ++i) acc[i] = make_float2(0.f, 0.f);
-      // scales for K block kb+1 are fetched while block kb is processed
-      const float* sap = tp.sa_t + grow;
-      float sa_n = sap[0];
-      float w0_n = __ldg(ws0), w1_n = __ldg(ws1);
-      for (int kb = 0; kb < (kFused ? nkb : p.num_kb); ++kb, ++kbg) {
-        const float s0 = sa_n * w0_n;
-        const float s1 = sa_n * w1_n;
-        if (kb + 1 < (kFused ? nkb : p.num_kb)) {
-          sa_n = sap[static_cast<size_t>(kb + 1) * p.rpad];
-          w0_n = __ldg(ws0 + kb + 1);
-          w1_n = __ldg(ws1 + kb + 1);
+      // weight-block scales of K block kb+2 are fetched while block kb is processed; the
+      // row scales come through the ring (this thread's is at its row's offset from the
+      // 16-byte boundary the producer copied from)
+      const int sofs = (c.row0 & 3) + trow;
+      float w0_n = __ldg(ws0 + kb0), w1_n = __ldg(ws1 + kb0);
+      float w0_n2 = 0.f, w1_n2 = 0.f;
+      if (kb0 + 1 < kb1) {
+        w0_n2 = __ldg(ws0 + kb0 + 1);
+        w1_n2 = __ldg(ws1 + kb0 + 1);
+      }
+      // the K block at which a pending count of the previous tile is taken
+      const int count_kb = kb0 + (kb1 - kb0 > 3 ? 3 : kb1 - kb0 - 1);
+      for (int kb = kb0; kb < kb1; ++kb, ++kbg) {
+        if (EPI == EPI_COMBINE && kb == count_kb && pend[1] > 0) {
+          // a few K blocks after they were issued the previous tile's reductions are done
+          combine_count(p, pend, trow, lane);
+        }
+        const int ss = kbg % kScaleSlots;
+        if (!mbar_wait(&S.sfull[ss], (kbg / kScaleSlots) & 1, abort_flag, p.status, p.wait_limit_ns)) {
+          ok = false;
+          break;
+        }
+        const float sa = S.sring[ss][sofs];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.sempty[ss]);
+        const float s0 = sa * w0_n;
+        const float s1 = sa * w1_n;
+        w0_n = w0_n2;
+        w1_n = w1_n2;
+        if (kb + 2 < kb1) {
+          w0_n2 = __ldg(ws0 + kb + 2);
+          w1_n2 = __ldg(ws1 + kb + 2);
         }
         const int b = kbg & 1;
         const uint32_t tph = (kbg >> 1) & 1;
@@ -580,10 +519,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tmem_wait_ld();
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) {
-            if (PAIR == 2) mbar_arrive_cluster(b ? tempty1 : tempty0);
-            else mbar_arrive(&S.tempty[b]);
-          }
+          if (lane == 0) mbar_arrive(&S.tempty[b]);
 #pragma unroll
           for (int i = 0; i < 16; ++i)
             acc[32 + i] = __ffma2_rn(make_float2(v[2 * i], v[2 * i + 1]), S1, acc[32 + i]);
@@ -594,19 +530,42 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       if (!ok) break;
 
-      if (swiglu) {
+      if (EPI == EPI_SWIGLU && splits > 1) {
+        // this unit's partial sum into G; the warp whose partial completes the tile's
+        // quadrant (two warps per split) finishes those 32 rows from G
+        if (valid) {
+          float* gr = p.g_ws + static_cast<size_t>(grow) * (2 * p.I) + c.nt * 128 + 64 * half;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) red_add_v4(gr + 4 * i, acc[2 * i].x, acc[2 * i].y, acc[2 * i + 1].x, acc[2 * i + 1].y);
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            red_add_v4(gr + p.I + 4 * i, acc[32 + 2 * i].x, acc[32 + 2 * i].y, acc[33 + 2 * i].x, acc[33 + 2 * i].y);
+        }
+        // one add per warp after every lane has fenced its reductions (two warps per split)
+        __threadfence();
+        __syncwarp();
+        int* cnt = p.g_cnt + tile * 4 + q;
+        int old = 0;
+        if (lane == 0) old = atomicAdd(cnt, 1);
+        old = __shfl_sync(0xffffffffu, old, 0);
+        if (old == 2 * splits - 1) {
+          __threadfence();
+          if (valid) split_swiglu_row(p, grow, c.nt);
+          __syncwarp();
+          if (lane == 0) *cnt = 0;          // zero again for the next call
+        }
+        continue;
+      }
+      if (EPI == EPI_SWIGLU) {
         // h = silu(g) * u on this thread's 64 channels; block amax shared with the partner
         // warp that holds the other 64 channels of the same rows
         float amax = 0.f;
-        // silu(g) = g / (1 + exp(-g)) with branch-free fast exp and division (g is
-        // clamped at -80, where silu is 0 to fp32 precision, so exp(-g) stays finite)
         float hv[64];
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           const float2 g = acc[i], u = acc[32 + i];
-          const float gx = fmaxf(g.x, -80.0f), gy = fmaxf(g.y, -80.0f);
-          hv[2 * i] = __fdividef(gx, 1.0f + __expf(-gx)) * u.x;
-          hv[2 * i + 1] = __fdividef(gy, 1.0f + __expf(-gy)) * u.y;
+          hv[2 * i] = silu_mul(g.x, u.x);
+          hv[2 * i + 1] = silu_mul(g.y, u.y);
           amax = fmaxf(amax, fmaxf(fabsf(hv[2 * i]), fabsf(hv[2 * i + 1])));
         }
         float* ax = &S.amax[titer & 1][0][0];
@@ -632,66 +591,106 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           for (int j = 0; j < 4; ++j) dst[j] = out[j];
           if (half == 0) p.sh_t[static_cast<size_t>(c.nt) * p.rpad + grow] = sc;
         }
-        if (kFused) {
-          // this warp's h rows and scales are stored: make them visible to the TMA loads
-          // and the epilogues of the W2 tiles of this m-tile
-          fence_proxy_async_global();
-          __syncwarp();
-          if (lane == 0) red_release_add(ready + c.mt, 1);
-        }
       } else {
-        // weighted combine: fp32 reductions into the token accumulator (kept in L2 with
-        // an evict-last hint), staged through shared memory so that each reduction covers
-        // 128 contiguous bytes of a row; combine_finalize_kernel turns the sums into bf16
-        int g = -1;
-        float wgt = 0.f;
-        if (valid) {
-          g = tp.row_token[grow];
-          wgt = tp.row_w[grow];
-        }
-        // the 32 rows go through the staging in two halves of 16; a reduction instruction
-        // then covers 4 rows x 128 contiguous bytes (8 lanes per row)
-        float* sw = stg + ew * 16 * kStgStride;
         const int col0 = c.nt * kBN + half * 128;
+        if (pend[1] > 0) combine_count(p, pend, trow, lane);
+        if (!p.fuse_final || c.e != p.G - 1) {
+          // weighted combine: this warp's 32 rows x 128 columns, times each row's top-K
+          // weight, go to the token accumulators as bulk reductions (one 512-byte row
+          // segment each). Eight lanes at a time fill one of the warp's two staging buffers
+          // and issue their rows; before a buffer is refilled, the lanes that issued from
+          // it last wait until the bulk engine has read it.
+          int g = -1;
+          float wgt = 0.f;
+          if (valid) {
+            g = p.row_token[grow];
+            wgt = p.row_w[grow];
+          }
+          uint8_t* wst = stg + ew * kStgWarpBytes;
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {          // 32 columns per chunk
+          for (int r8 = 0; r8 < 4; ++r8) {
+            uint8_t* buf = wst + (r8 & 1) * kStgBufBytes;
+            if ((lane >> 3) == ((r8 + 2) & 3)) bulk_wait_read_all();
+            __syncwarp();
+            if ((lane >> 3) == r8) {
+              float* row = reinterpret_cast<float*>(buf + (lane & 7) * kStgRowBytes);
 #pragma unroll
-          for (int hr = 0; hr < 2; ++hr) {
-            if ((lane >> 4) == hr) {
-#pragma unroll
-              for (int j = 0; j < 8; ++j) {
-                const float2 a = acc[16 * ch + 2 * j], bb = acc[16 * ch + 2 * j + 1];
-                *reinterpret_cast<float4*>(sw + (lane & 15) * kStgStride + 4 * j) =
+              for (int i = 0; i < 32; ++i) {
+                const float2 a = acc[2 * i], bb = acc[2 * i + 1];
+                *reinterpret_cast<float4*>(row + 4 * i) =
                     make_float4(a.x * wgt, a.y * wgt, bb.x * wgt, bb.y * wgt);
               }
+              fence_proxy_async_shared();
+              if (g >= 0)
+                bulk_reduce_add_f32(p.acc + static_cast<size_t>(g) * p.H + col0, row, 512, pol_acc);
+              bulk_commit();
+            }
+          }
+          if (p.fuse_final) {
+            __syncwarp();
+            if (lane == 0) {
+              pend[0] = c.row0;
+              pend[1] = c.rows;
+              pend[2] = c.nt;
             }
             __syncwarp();
+          }
+        } else {
+          // the shared expert's tile of token block tb (its rows are the tokens 128 tb ..
+          // 128 tb + 127, weight 1): once the routed rows of the block are in, add this
+          // row to the accumulated sum, write bf16 into the token's slab row, clear the sum
+          const int tb = c.mt - S.mtile[p.G - 1];
+          const int* cnt = p.blk_cnt + static_cast<size_t>(tb) * p.n_tiles + c.nt;
+          const int target = p.blk_need[tb];
+          int got = 1;
+          if (lane == 0) got = wait_count(cnt, target, abort_flag, p.status, p.wait_limit_ns);
+          got = __shfl_sync(0xffffffffu, got, 0);
+          if (!got) {
+            ok = false;
+            break;
+          }
+          ld_acquire(cnt);
+          if (valid) {
+            const int g = 128 * tb + trow;
+            const int mt = p.tok_mt[g];
+            float* arow = p.acc + static_cast<size_t>(g) * p.H + col0;
+            uint4* yrow = reinterpret_cast<uint4*>(ytab.y[mt >> 24] + static_cast<size_t>(mt & 0xFFFFFF) * p.H + col0);
 #pragma unroll
-            for (int r4 = 0; r4 < 4; ++r4) {
-              const int rl = r4 * 4 + (lane >> 3);
-              const int cc = (lane & 7) * 4;
-              const int gg = __shfl_sync(0xffffffffu, g, 16 * hr + rl);
-              const float4 v = *reinterpret_cast<const float4*>(sw + rl * kStgStride + cc);
-              if (gg >= 0)
-                red_add_v4_hint(tp.acc + static_cast<size_t>(gg) * tp.H + col0 + 32 * ch + cc, v.x,
-                                v.y, v.z, v.w, pol_acc);
+            for (int h4 = 0; h4 < 4; ++h4) {      // 32 columns at a time
+              float4 a[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) a[i] = __ldcg(reinterpret_cast<const float4*>(arow + 32 * h4 + 4 * i));
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const float4 u = a[2 * i], v = a[2 * i + 1];
+                const float2 x0 = acc[16 * h4 + 4 * i], x1 = acc[16 * h4 + 4 * i + 1];
+                const float2 x2 = acc[16 * h4 + 4 * i + 2], x3 = acc[16 * h4 + 4 * i + 3];
+                uint4 o;
+                o.x = pack_bf16x2(u.x + x0.x, u.y + x0.y);
+                o.y = pack_bf16x2(u.z + x1.x, u.w + x1.y);
+                o.z = pack_bf16x2(v.x + x2.x, v.y + x2.y);
+                o.w = pack_bf16x2(v.z + x3.x, v.w + x3.y);
+                yrow[4 * h4 + i] = o;
+              }
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                __stcg(reinterpret_cast<float4*>(arow + 32 * h4 + 4 * i), make_float4(0.f, 0.f, 0.f, 0.f));
             }
-            __syncwarp();
           }
         }
       }
     }
+    if (EPI == EPI_COMBINE && ok && pend[1] > 0) combine_count(p, pend, trow, lane);
+    // every bulk reduction issued by this thread has been performed before the CTA exits
+    if (EPI == EPI_COMBINE) bulk_wait_all();
   }
 
   tc_fence_before();
   __syncthreads();
-  // neither CTA of a pair leaves while the other may still signal its barriers
-  if (PAIR == 2) cluster_sync();
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    if (PAIR == 2) tmem_dealloc_pair(tmem_base, kTmemCols);
-    else tmem_dealloc(tmem_base, kTmemCols);
+    tmem_dealloc(tmem_base, kTmemCols);
   }
 }
 

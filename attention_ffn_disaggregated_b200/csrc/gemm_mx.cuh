@@ -1,4 +1,4 @@
-// W13 grouped GEMM on the tensor core's block-scale path (tiling 5), for inputs whose
+// W13 grouped GEMM on the tensor core's block-scale path (tiling 2), for inputs whose
 // block scales are all powers of two: FastAFD, "Methodology / System Design", item 1
 // (block-FP8 expert precision) and item 3 (block-FP8 grouped GEMMs, activation).
 //
@@ -36,7 +36,7 @@ constexpr uint32_t kSfImage = 512;                 // bytes per 128 rows x one 1
 constexpr uint32_t kSfStage = 3 * kSfImage;        // A rows, W13 gate block, W13 up block
 constexpr uint32_t kMxSfCol = 256;                 // first factor column in TMEM
 constexpr uint32_t kMxSfCols = 16;                 // factor columns per stage
-constexpr size_t kMxTiles = static_cast<size_t>(kMxStages) * Tiling<1>::kStageBytes;
+constexpr size_t kMxTiles = static_cast<size_t>(kMxStages) * kStageBytes;
 static_assert(kMxSfCol + kMxStages * kMxSfCols <= kTmemCols, "factor columns exceed TMEM");
 
 struct alignas(16) MxSmem {
@@ -98,7 +98,7 @@ __global__ void __launch_bounds__(128) mx_act_sf_kernel(const int32_t* __restric
   const int i = threadIdx.x;
   for (int u = blockIdx.x; u < n_img; u += gridDim.x) {
     const int mt = u / num_kb, kb = u - mt * num_kb;
-    const TileCoord c = decode_tile<1>(mt, 1, mtile_off, G, group_off, 0);
+    const TileCoord c = decode_tile(mt, 1, 0, mtile_off, G, group_off);
     bool bad;
     const uint32_t e = ue8m0_of(sa_t[static_cast<size_t>(kb) * rpad + c.row0 + i], bad);
     if (bad && i < c.rows) atomicOr(status, AFD_STATUS_BAD_SCALE);
@@ -110,7 +110,6 @@ __global__ void __launch_bounds__(128) mx_act_sf_kernel(const int32_t* __restric
 __global__ void __launch_bounds__(kGemmThreads, 1)
     w13_mx_kernel(const __grid_constant__ GemmParams p, const __grid_constant__ CUtensorMap tm_a,
                   const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ MxArgs mx) {
-  using TL = Tiling<1>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -159,7 +158,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int it = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
-        const TileCoord c = decode_tile<1>(tile, p.n_tiles, S.mtile, p.G, p.group_off, 0);
+        const TileCoord c = decode_tile(tile, p.n_tiles, 0, S.mtile, p.G, p.group_off);
         const int brow0 = c.nt * 128;              // gate block
         const int brow1 = p.I + c.nt * 128;        // up block
         const uint8_t* fa = mx.sfa + static_cast<size_t>(c.mt) * nkb * kSfImage;
@@ -173,12 +172,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             break;
           }
           uint8_t* a = sA + s * kABytes;
-          uint8_t* b = sB + s * TL::kBBytes;
+          uint8_t* b = sB + s * kBBytes;
           uint8_t* f = sF + s * kSfStage;
-          mbar_arrive_expect_tx(&S.full[s], TL::kStageBytes + kSfStage);
+          mbar_arrive_expect_tx(&S.full[s], kStageBytes + kSfStage);
           tma_load_2d(a, &tm_a, &S.full[s], kb * kBK, c.row0, pol);
           tma_load_3d(b, &tm_b, &S.full[s], kb * kBK, brow0, c.e, pol);
-          tma_load_3d(b + TL::kBBytes / 2, &tm_b, &S.full[s], kb * kBK, brow1, c.e, pol);
+          tma_load_3d(b + kBBytes / 2, &tm_b, &S.full[s], kb * kBK, brow1, c.e, pol);
           bulk_load(f, fa + static_cast<size_t>(kb) * kSfImage, kSfImage, &S.full[s]);
           bulk_load(f + kSfImage, fg + static_cast<size_t>(kb) * kSfImage, kSfImage, &S.full[s]);
           bulk_load(f + 2 * kSfImage, fu + static_cast<size_t>(kb) * kSfImage, kSfImage, &S.full[s]);
@@ -216,7 +215,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tmem_cp_32x128b_x4(tsfb, sdesc_rows16(f + kSfImage));           // columns 0..127
           tmem_cp_32x128b_x4(tsfb + 4, sdesc_rows16(f + 2 * kSfImage));   // columns 128..255
           const uint64_t a0 = sdesc_k_sw128(smem_u32(sA + s * kABytes));
-          const uint64_t b0 = sdesc_k_sw128(smem_u32(sB + s * TL::kBBytes));
+          const uint64_t b0 = sdesc_k_sw128(smem_u32(sB + s * kBBytes));
 #pragma unroll
           for (int k = 0; k < kBK / 32; ++k)
             umma_mx_e4m3(tmem_base, a0 + 2 * k, b0 + 2 * k, idesc, tsfa, tsfb, (kb | k) != 0 ? 1u : 0u);
@@ -243,7 +242,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     int titer = 0;
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x, ++titer) {
-      const TileCoord c = decode_tile<1>(tile, p.n_tiles, S.mtile, p.G, p.group_off, 0);
+      const TileCoord c = decode_tile(tile, p.n_tiles, 0, S.mtile, p.G, p.group_off);
       const int grow = c.row0 + trow;
       const bool valid = trow < c.rows;
       int got = 1;

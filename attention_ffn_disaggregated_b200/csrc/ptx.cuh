@@ -1,6 +1,6 @@
 // Device primitives for sm_100a, written against the PTX ISA: mbarriers with bounded
-// waits, TMA tile loads (no cluster multicast anywhere), tcgen05 TMEM allocation, MMA,
-// commit and loads, and small warp helpers.
+// waits, TMA tile loads and bulk copies / reductions (no cluster multicast anywhere),
+// tcgen05 TMEM allocation, MMA, commit and loads, and small warp helpers.
 #pragma once
 
 #include <cstdint>
@@ -106,20 +106,6 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* m, uin
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
       ".L2::cache_hint [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)), "r"(x), "r"(y), "l"(policy)
-      : "memory");
-}
-
-// Four rows of a 2D map whose box is {columns, 1}: rows y0..y3 at column x land in four
-// consecutive box-sized rows at dst (swizzled by their shared-memory address like a
-// tiled load of the same four rows).
-__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* m, uint64_t* bar, int32_t x,
-                                            int32_t y0, int32_t y1, int32_t y2, int32_t y3,
-                                            uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cta.global.tile::gather4.mbarrier::complete_tx::bytes"
-      ".cta_group::1.L2::cache_hint [%0], [%1, {%3, %4, %5, %6, %7}], [%2], %8;" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)), "r"(x), "r"(y0), "r"(y1), "r"(y2),
-      "r"(y3), "l"(policy)
       : "memory");
 }
 
@@ -285,150 +271,43 @@ __device__ __forceinline__ void tmem_wait_ld() {
 }
 
 // ------------------------------------------------------------------------------------
-// CTA pairs (clusters of two): one leader issues MMAs that span both CTAs' shared
-// memory and tensor memory (cta_group::2). No cluster multicast is used: a load or a
-// commit that must reach the other CTA names that CTA's barrier explicitly.
-// ------------------------------------------------------------------------------------
-__device__ __forceinline__ uint32_t cluster_ctarank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-
-// Address of the same shared-memory offset in CTA `rank` of this cluster.
-__device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
-  return r;
-}
-
-__device__ __forceinline__ void cluster_sync() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
-                   : "memory");
-}
-
-// arrive on an mbarrier that may live in the other CTA of the cluster
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
-               : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// Bounded wait with cluster-scope acquire (for barriers the other CTA arrives on).
-__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity,
-                                                  volatile int* abort_flag, int* status,
-                                                  uint64_t limit_ns) {
-  const uint32_t a = smem_u32(bar);
-  if (mbar_try_wait_cluster(a, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  uint32_t n = 0;
-  while (true) {
-    if (mbar_try_wait_cluster(a, parity)) return true;
-    if ((++n & 63u) == 0) {
-      if (*abort_flag) return false;
-      if (globaltimer_ns() - t0 > limit_ns) {
-        *abort_flag = 1;
-        atomicOr(status, AFD_STATUS_TIMEOUT);
-        return false;
-      }
-    }
-  }
-}
-
-// TMA tile loads issued by either CTA of a pair whose completion is counted on the
-// leader's mbarrier (cluster address `bar_cluster`); no multicast.
-__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* m, uint32_t bar_cluster,
-                                                 int32_t x, int32_t y, uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-      ".L2::cache_hint [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(m)), "r"(bar_cluster), "r"(x), "r"(y), "l"(policy)
-      : "memory");
-}
-
-__device__ __forceinline__ void tma_load_3d_pair(void* dst, const CUtensorMap* m, uint32_t bar_cluster,
-                                                 int32_t x, int32_t y, int32_t z, uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-      ".L2::cache_hint [%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(m)), "r"(bar_cluster), "r"(x), "r"(y), "r"(z), "l"(policy)
-      : "memory");
-}
-
-__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
-  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                   smem_u32(dst_smem)),
-               "r"(ncols)
-               : "memory");
-}
-
-__device__ __forceinline__ void tmem_relinquish_pair() {
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
-}
-
-__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
-  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
-               : "memory");
-}
-
-// One MMA over the pair: A rows split between the two CTAs (M = 256), B rows (N) split
-// between their shared memories; each CTA's TMEM receives its own 128 rows.
-__device__ __forceinline__ void umma_e4m3_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
-                                               uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// Arrive on the mbarrier at cluster address `bar_cluster` once the pair MMAs this thread
-// issued so far have completed.
-__device__ __forceinline__ void umma_commit_pair(uint32_t bar_cluster) {
-  asm volatile(
-      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-          bar_cluster)
-      : "memory");
-}
-
-// ------------------------------------------------------------------------------------
 // misc
 // ------------------------------------------------------------------------------------
-__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-
+// fp32 vector reduction into global memory (relaxed, performed at L2)
 __device__ __forceinline__ void red_add_v4(float* gaddr, float a, float b, float c, float d) {
   asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(gaddr), "f"(a), "f"(b),
                "f"(c), "f"(d)
                : "memory");
 }
 
-// fp32 vector reduction into global memory with an L2 cache-eviction hint
-__device__ __forceinline__ void red_add_v4_hint(float* gaddr, float a, float b, float c, float d,
-                                                uint64_t policy) {
-  asm volatile("red.global.add.L2::cache_hint.v4.f32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(gaddr),
-               "f"(a), "f"(b), "f"(c), "f"(d), "l"(policy)
-               : "memory");
+// Bulk reduction, shared -> global, performed by the bulk-copy engine: `bytes` (a multiple
+// of 16) of fp32 at `src` are added to `dst` (both 16-byte aligned), with an L2 eviction
+// hint. Completion is tracked per thread in bulk groups (bulk_commit / bulk_wait_*).
+__device__ __forceinline__ void bulk_reduce_add_f32(float* dst, const void* src, uint32_t bytes,
+                                                    uint64_t policy) {
+  asm volatile(
+      "cp.reduce.async.bulk.global.shared::cta.bulk_group.L2::cache_hint.add.f32 [%0], [%1], %2, %3;" ::"l"(
+          dst),
+      "r"(smem_u32(src)), "r"(bytes), "l"(policy)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// wait until every bulk group of this thread has finished reading its shared-memory source
+__device__ __forceinline__ void bulk_wait_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// wait until every bulk group of this thread has been performed
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+// make this thread's generic-proxy shared-memory stores visible to the bulk-copy engine
+__device__ __forceinline__ void fence_proxy_async_shared() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-// Cross-CTA readiness counters (release / acquire at GPU scope). A writer whose data
-// will be read by TMA (the async proxy) fences its generic stores to that proxy first.
-__device__ __forceinline__ void fence_proxy_async_global() {
-  asm volatile("fence.proxy.async.global;" ::: "memory");
-}
+// Cross-CTA counters (release / acquire at GPU scope).
 __device__ __forceinline__ void red_release_add(int* addr, int v) {
   asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(addr), "r"(v) : "memory");
 }
@@ -445,7 +324,7 @@ __device__ __forceinline__ bool wait_count(const int* addr, int target, volatile
   const uint64_t t0 = globaltimer_ns();
   uint32_t n = 0;
   while (true) {
-    __nanosleep(100);
+    __nanosleep(64);
     if (ld_acquire(addr) >= target) return true;
     if ((++n & 15u) == 0) {
       if (*abort_flag) return false;
@@ -457,9 +336,10 @@ __device__ __forceinline__ bool wait_count(const int* addr, int target, volatile
     }
   }
 }
-
-__device__ __forceinline__ float4 ld_cg_f4(const float* p) {
-  return __ldcg(reinterpret_cast<const float4*>(p));
+// order this thread's completed bulk (async-proxy) global writes before its later
+// generic-proxy operations
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -39,12 +39,16 @@ struct RouteParams {
   int32_t* group_count;   // [G]
   int32_t* group_off;     // [G+1]
   int32_t* mtile_off;     // [G+1] 128-row m-tiles
-  int32_t* mtile2_off;    // [G+1] 256-row m-tiles (CTA-pair tiling); may be null
   int* scan_ticket;       // zero between calls: route_count runs the scan; null: separate
-  int32_t* ready;         // [m-tiles] fused GEMM readiness counters, zeroed by the scan; may be null
-  int tiling;             // as set on the plan: 0 (default, = 1) .. 5; -1: routing only
+  int tiling;             // as set on the plan: 0 (default, = 1) .. 2; -1: routing only
   int32_t* tok_mt;        // [Tmax] (slab << 24) | row
   int32_t* tok_need;      // [Tmax] contributions this GPU adds to the token
+  // fused combine (layers with a shared expert; null otherwise): per 128-token block, the
+  // count the down projection's routed tiles reach (two per routed row: one per epilogue
+  // half), and the per (block, 256-column tile) counters they add to, zeroed here
+  int32_t* blk_need;      // [2 * num_chunks]
+  int32_t* blk_cnt;       // [2 * num_chunks][n_ctiles]
+  int n_ctiles;
   int32_t* pos;           // [Tmax*K]
   int32_t* row_token;     // [rpad]
   int32_t* row_k;         // [rpad]
@@ -150,36 +154,29 @@ __device__ void route_scan_body(const RouteParams& p, int T, int* s_warp) {
   __syncthreads();
   if (p.S && threadIdx.x == 0) p.group_count[p.El] = T;
   __syncthreads();
-  int base_rows = 0, base_tiles = 0, base_tiles2 = 0;
+  int base_rows = 0, base_tiles = 0;
   for (int g0 = 0; g0 < p.G; g0 += blockDim.x) {
     const int g = g0 + threadIdx.x;
     const int cnt = g < p.G ? p.group_count[g] : 0;
-    int tot_rows, tot_tiles, tot_tiles2;
+    int tot_rows, tot_tiles;
     const int ex_rows = block_exclusive_scan(cnt, s_warp, &tot_rows);
     const int ex_tiles = block_exclusive_scan((cnt + kTileM - 1) / kTileM, s_warp, &tot_tiles);
-    const int ex_tiles2 =
-        block_exclusive_scan((cnt + 2 * kTileM - 1) / (2 * kTileM), s_warp, &tot_tiles2);
     if (g < p.G) {
       p.group_off[g] = base_rows + ex_rows;
       p.mtile_off[g] = base_tiles + ex_tiles;
-      if (p.mtile2_off) p.mtile2_off[g] = base_tiles2 + ex_tiles2;
     }
     base_rows += tot_rows;
     base_tiles += tot_tiles;
-    base_tiles2 += tot_tiles2;
   }
   if (threadIdx.x == 0) {
     p.group_off[p.G] = base_rows;
     p.mtile_off[p.G] = base_tiles;
-    if (p.mtile2_off) p.mtile2_off[p.G] = base_tiles2;
     p.info[1] = base_rows;
     p.info[2] = base_tiles;
     // the tiling this call runs (the host launches only its kernels); 0 for routing
     // without a layer
     p.info[3] = p.tiling < 0 ? 0 : (p.tiling == 0 ? 1 : p.tiling);
   }
-  if (p.ready)
-    for (int i = threadIdx.x; i < base_tiles; i += blockDim.x) p.ready[i] = 0;
 }
 
 // 2 as its own launch (one block of 1024 threads).
@@ -204,6 +201,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_count_kernel(
   for (int e = threadIdx.x; e < p.El; e += blockDim.x) s_hist[e] = 0;
   __syncthreads();
   const int g = blockIdx.x * kChunkTokens + threadIdx.x;
+  int routed = 0;
   if (g < T) {
     const int m = find_slab(s_base, p.M, g);
     const int t = g - s_base[m];
@@ -217,7 +215,24 @@ __global__ void __launch_bounds__(kRouteThreads) route_count_kernel(
       if (mask >> k & 1u) atomicAdd(&s_hist[le[k]], 1);
     p.tok_mt[g] = (m << 24) | t;
     p.tok_need[g] = __popc(mask) + p.S;
+    routed = __popc(mask);
     if (bad) atomicOr(p.status, AFD_STATUS_BAD_ROUTING);
+  }
+  if (p.blk_need) {
+    // this CTA's two 128-token blocks: their targets and zeroed counters
+    static_assert(kChunkTokens == 256 && kRouteWarps == 8, "two 128-token blocks per routing CTA");
+    __shared__ int s_bn[kRouteWarps];
+    int v = routed;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if ((threadIdx.x & 31) == 0) s_bn[threadIdx.x >> 5] = v;
+    const size_t tb0 = static_cast<size_t>(blockIdx.x) * 2;
+    for (int i = threadIdx.x; i < 2 * p.n_ctiles; i += blockDim.x) p.blk_cnt[tb0 * p.n_ctiles + i] = 0;
+    __syncthreads();
+    if (threadIdx.x < 2) {
+      const int* w = s_bn + 4 * threadIdx.x;
+      p.blk_need[tb0 + threadIdx.x] = 2 * (w[0] + w[1] + w[2] + w[3]);
+    }
   }
   __syncthreads();
   int32_t* out = p.chunk_hist + static_cast<size_t>(blockIdx.x) * max(p.El, 1);
@@ -391,20 +406,6 @@ __global__ void __launch_bounds__(kRouteThreads) gather_rows_kernel(
       }
       if (shared_row >= 0) dcol[shared_row] = sc;
     }
-  }
-}
-
-// 4b. when the W13 GEMM fetches its A rows from the slabs itself, only the per-128 scales
-// move into expert order: one thread per row, so that each K block's 32 consecutive rows
-// are written with one coalesced store per warp.
-__global__ void __launch_bounds__(kRouteThreads) gather_scales_kernel(
-    const __grid_constant__ RouteParams p, const __grid_constant__ SlabTable slabs) {
-  const int R = p.info[1];
-  const int KB = p.H / AFD_QBLOCK;
-  for (int r = blockIdx.x * blockDim.x + threadIdx.x; r < R; r += gridDim.x * blockDim.x) {
-    const int mt = p.tok_mt[p.row_token[r]];
-    const float* __restrict__ src = slabs.xs[mt >> 24] + static_cast<size_t>(mt & 0xFFFFFF) * KB;
-    for (int kb = 0; kb < KB; ++kb) p.sa_t[static_cast<size_t>(kb) * p.rpad + r] = __ldg(src + kb);
   }
 }
 

@@ -46,6 +46,16 @@ class PlanInfo(ctypes.Structure):
                 ("num_sms", c_int32), ("workspace_bytes", c_int64)]
 
 
+class BoundSlabs:
+    """A slab set marshalled by FfnLayer.bind: the descriptor array and the counts pointer
+    (the tensors are kept referenced)."""
+
+    def __init__(self, descs, counts, keep):
+        self.descs = descs
+        self.counts = counts
+        self._keep = keep
+
+
 class AfdError(RuntimeError):
     def __init__(self, code: int, what: str):
         super().__init__(f"{what}: {STATUS_NAMES.get(code, code)}")
@@ -79,7 +89,7 @@ def lib() -> ctypes.CDLL:
         "afd_ffn_inject_stall": (c_int32, [P, c_int32]),
         "afd_ffn_set_tiling": (c_int32, [P, c_int32]),
         "afd_ffn_get_tiling": (c_int32, [P, P, POINTER(c_int32)]),
-        "afd_ffn_kernels_per_layer": (c_int32, []),
+        "afd_ffn_kernels_per_layer": (c_int32, [P]),
         "afd_ffn_route_noalloc": (c_int32, [POINTER(Config), POINTER(SlabDesc), P, P, P, P, P, P, P, P,
                                             P, P]),
         "afd_status_string": (c_char_p, [c_int32]),
@@ -146,7 +156,6 @@ class FfnLayer:
         self.plan = h
         self.info = PlanInfo()
         L.afd_ffn_get_info(self.plan, ctypes.byref(self.info))
-        self._descs = (SlabDesc * num_slabs)()
 
     def close(self):
         if getattr(self, "plan", None):
@@ -159,16 +168,23 @@ class FfnLayer:
         except Exception:
             pass
 
-    def __call__(self, slabs: Sequence, counts, stream=None) -> None:
-        """slabs: sequence of objects with .x .x_scale .topk_ids .topk_weights .y CUDA tensors."""
+    def bind(self, slabs: Sequence, counts) -> "BoundSlabs":
+        """Marshal a slab set once (its device pointers, checked) for repeated calls: a
+        serving loop whose receive buffers are fixed passes the result to __call__ instead
+        of the slabs, so that a call costs one C call on the host."""
         if len(slabs) != self.num_slabs:
             raise ValueError("expected %d slabs" % self.num_slabs)
+        descs = (SlabDesc * self.num_slabs)()
         for i, s in enumerate(slabs):
-            self._descs[i] = SlabDesc(_ptr(s.x, "x"), _ptr(s.x_scale, "x_scale"),
-                                      _ptr(s.topk_ids, "topk_ids"),
-                                      _ptr(s.topk_weights, "topk_weights"), _ptr(s.y, "y"))
-        rc = lib().afd_ffn_layer(self.plan, self._descs, c_void_p(_ptr(counts, "counts")),
-                                 c_void_p(_stream_handle(stream)))
+            descs[i] = SlabDesc(_ptr(s.x, "x"), _ptr(s.x_scale, "x_scale"), _ptr(s.topk_ids, "topk_ids"),
+                                _ptr(s.topk_weights, "topk_weights"), _ptr(s.y, "y"))
+        return BoundSlabs(descs, c_void_p(_ptr(counts, "counts")), (slabs, counts))
+
+    def __call__(self, slabs, counts=None, stream=None) -> None:
+        """slabs: a sequence of objects with .x .x_scale .topk_ids .topk_weights .y CUDA
+        tensors and counts a device int32 tensor, or a BoundSlabs from bind() (counts None)."""
+        b = slabs if isinstance(slabs, BoundSlabs) else self.bind(slabs, counts)
+        rc = lib().afd_ffn_layer(self.plan, b.descs, b.counts, c_void_p(_stream_handle(stream)))
         if rc != AFD_OK:
             raise AfdError(rc, "afd_ffn_layer")
 
@@ -227,17 +243,16 @@ class FfnLayer:
             raise AfdError(rc, "afd_ffn_set_wait_limit")
 
     def set_tiling(self, tiling: int):
-        """0: default (1); 1: single-CTA tiles; 2: CTA-pair tiles; 3: single-CTA tiles with the
-        W13 rows gathered from the slabs by TMA (no expert-ordered row copy); 4: W13 and W2 in
-        one persistent launch; 5: W13 on the block-scale MMA path, for inputs whose
-        activation and W13 block scales are all powers of two (the first selection builds
-        the W13 factor images and synchronises the device)."""
+        """0: default (1); 1: software-promoted block-FP8 GEMMs (any fp32 block scales); 2: W13
+        on the block-scale MMA path, for inputs whose activation and W13 block scales are all
+        powers of two (the first selection builds and checks the W13 factor images and
+        synchronises the device; weights with other scales are refused)."""
         rc = lib().afd_ffn_set_tiling(self.plan, int(tiling))
         if rc != AFD_OK:
             raise AfdError(rc, "afd_ffn_set_tiling")
 
     def tiling(self, stream=None) -> int:
-        """Tiling (1 to 5) the last layer call used."""
+        """Tiling (1 or 2) the last layer call used."""
         t = c_int32(0)
         rc = lib().afd_ffn_get_tiling(self.plan, c_void_p(_stream_handle(stream)), ctypes.byref(t))
         if rc != AFD_OK:
@@ -248,8 +263,9 @@ class FfnLayer:
         lib().afd_ffn_inject_stall(self.plan, 1 if enable else 0)
 
 
-def kernels_per_layer() -> int:
-    return lib().afd_ffn_kernels_per_layer()
+def kernels_per_layer(layer: "FfnLayer") -> int:
+    """Kernel launches one call of `layer` makes with its current tiling."""
+    return lib().afd_ffn_kernels_per_layer(layer.plan)
 
 
 def route_noalloc(shape, slabs: Sequence, counts, stream=None) -> dict:

@@ -45,14 +45,18 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-tokens", type=int, default=64)
-    ap.add_argument("--tiling", type=int, default=0, choices=[0, 1, 2, 3, 4, 5],
-                    help="GEMM tiling (afd_ffn_set_tiling); 0 = the library default")
+    ap.add_argument("--tiling", type=int, default=0, choices=[0, 1, 2],
+                    help="GEMM tiling (afd_ffn_set_tiling); 0 = the library default (1), "
+                         "2 = block-scale W13 (power-of-two scales only)")
     ap.add_argument("--graph", action="store_true",
                     help="time replays of the layer captured in a CUDA graph")
     ap.add_argument("--sweep", action="store_true",
                     help="batch / fan-in sweep at the DeepSeek-V3 share shape: one line per cell")
     ap.add_argument("--sweep-filter", default="",
                     help="only sweep cells whose name contains this string")
+    ap.add_argument("--quick", action="store_true",
+                    help="device-timed steps only (no graph replay, end-to-end, ping-pong or CPU "
+                         "baseline passes); for profiling runs")
     return ap.parse_args()
 
 
@@ -81,17 +85,34 @@ def workload_bytes_flops(inp, routing_counts):
     return bytes_, flops, R, active
 
 
-def source_hash():
+# The source files each timed stage's kernel is compiled from (its traffic record is
+# stale once one of them changes).
+CSRC = "attention_ffn_disaggregated_b200/csrc/"
+KERNEL_SOURCES = {
+    "gemm13_swiglu": [CSRC + "gemm.cuh", CSRC + "ptx.cuh", CSRC + "route.cuh", "include/afd_ffn.h"],
+    "gemm2_combine": [CSRC + "gemm.cuh", CSRC + "ptx.cuh", CSRC + "route.cuh", "include/afd_ffn.h"],
+    "combine_finalize": [CSRC + "gemm.cuh", CSRC + "ptx.cuh", CSRC + "route.cuh", "include/afd_ffn.h"],
+    "gather_rows": [CSRC + "route.cuh", CSRC + "ptx.cuh", "include/afd_ffn.h"],
+    "route_count": [CSRC + "route.cuh", CSRC + "ptx.cuh", "include/afd_ffn.h"],
+    "route_scatter": [CSRC + "route.cuh", CSRC + "ptx.cuh", "include/afd_ffn.h"],
+}
+
+
+def source_hash(kernel: str = "") -> str:
+    """Hash of the files `kernel` is built from (of the whole CUDA tree without a name)."""
+    files = KERNEL_SOURCES.get(kernel)
+    if files is None:
+        files = [os.path.join(d, f) for d in (CSRC.rstrip("/"), "include")
+                 for f in sorted(os.listdir(os.path.join(ROOT, d)))]
     h = hashlib.sha256()
-    for d in ("attention_ffn_disaggregated_b200/csrc", "include"):
-        for f in sorted(os.listdir(os.path.join(ROOT, d))):
-            h.update(open(os.path.join(ROOT, d, f), "rb").read())
+    for f in files:
+        h.update(open(os.path.join(ROOT, f), "rb").read())
     return h.hexdigest()[:16]
 
 
 def profiled_traffic(kernel: str, workload: str):
-    """DRAM bytes per launch recorded by ncu for this kernel source on this workload (None
-    if stale, missing or captured on another workload)."""
+    """DRAM bytes per launch recorded by ncu for this kernel's sources on this workload
+    (None if stale, missing or captured on another workload)."""
     p = os.path.join(ROOT, "profiles", f"{kernel}_traffic.txt")
     if not os.path.exists(p):
         return None
@@ -100,7 +121,7 @@ def profiled_traffic(kernel: str, workload: str):
         if ":" in line and not line.startswith("#"):
             k, v = line.split(":", 1)
             kv[k.strip()] = v.strip()
-    if kv.get("source_sha") != source_hash() or kv.get("workload") != workload:
+    if kv.get("source_sha") != source_hash(kernel) or kv.get("workload") != workload:
         return None
     try:
         return float(kv["dram_bytes_per_launch_full"])
@@ -240,17 +261,18 @@ def time_layer(layer, slabs, counts, flush, steps, warmup, graph=False):
     """Device time of `steps` layer calls (ms each), L2 flushed before every call."""
     import torch
     stream = torch.cuda.current_stream()
-    run = lambda: layer(slabs, counts)
+    bound = layer.bind(slabs, counts)
+    run = lambda: layer(bound)
     g = None
     if graph:
         layer.set_timing(False)          # no per-kernel events inside the captured graph
         side = torch.cuda.Stream()
         with torch.cuda.stream(side):
-            layer(slabs, counts)
+            layer(bound)
         torch.cuda.synchronize()
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=side):
-            layer(slabs, counts)
+            layer(bound)
         run = g.replay
     for _ in range(warmup):
         flush.zero_()
@@ -304,6 +326,8 @@ def time_e2e(layer, inp, slab_sets, count_sets, flush, steps, warmup):
         for s, yh, n in zip(slab_sets[b], y_h[b], ns):
             yh[:n].copy_(s.y[:n], non_blocking=True)
 
+    bound = [layer.bind(slab_sets[b], count_sets[b]) for b in range(2)]
+
     def serial(n_steps):
         total = 0.0
         for _ in range(n_steps):
@@ -311,7 +335,7 @@ def time_e2e(layer, inp, slab_sets, count_sets, flush, steps, warmup):
             e0.record(comp)
             upload(0)
             flush.zero_()
-            layer(slab_sets[0], count_sets[0])
+            layer(bound[0])
             download(0)
             e1.record(comp)
             e1.synchronize()
@@ -337,7 +361,7 @@ def time_e2e(layer, inp, slab_sets, count_sets, flush, steps, warmup):
             if down_done[b] is not None:
                 comp.wait_event(down_done[b])         # set b's previous outputs are on the host
             flush.zero_()
-            layer(slab_sets[b], count_sets[b])
+            layer(bound[b])
             comp_done[b] = torch.cuda.Event()
             comp_done[b].record(comp)
             with torch.cuda.stream(down):
@@ -356,6 +380,66 @@ def time_e2e(layer, inp, slab_sets, count_sets, flush, steps, warmup):
     pipelined(warmup)
     t_pipe = pipelined(steps)
     return t_serial / steps, t_pipe / steps, h2d, d2h
+
+
+def time_ping_pong(inp, dev_w, slabs, flush, steps, warmup, tiling):
+    """Device time (ms) of one step of two ping-pong microbatches (FastAFD, "Methodology /
+    System Design", item 4, k = 2): each slab's valid rows are split into a first and a
+    second half; microbatch A (the first halves) and B (the rest) are served by two plans
+    over the same weights, on two streams, concurrently."""
+    import torch
+    from attention_ffn_disaggregated_b200 import FfnLayer
+    from attention_ffn_disaggregated_b200.device import DeviceSlab
+    ns = [int(n) for n in inp.counts]
+    cap = inp.capacity
+    na = [(n + 1) // 2 for n in ns]
+    # B's slabs are views that start at A's end: same buffers, capacity cap - na
+    cap_b = max(1, cap - max(na))
+    halves = []
+    for part in range(2):
+        views, cnt = [], []
+        for s, n, a in zip(slabs, ns, na):
+            off = 0 if part == 0 else a
+            rows = (cap if part == 0 else cap_b)
+            v = lambda t: t[off:off + rows] if off + rows <= t.shape[0] else t[off:]
+            views.append(DeviceSlab(v(s.x), v(s.x_scale), v(s.topk_ids), v(s.topk_weights), v(s.y)))
+            cnt.append(a if part == 0 else n - a)
+        halves.append((views, torch.tensor(cnt, dtype=torch.int32, device="cuda")))
+    plans = [FfnLayer(inp.shape, len(slabs), cap, *dev_w),
+             FfnLayer(inp.shape, len(slabs), cap_b, *dev_w)]
+    for pl in plans:
+        pl.set_tiling(tiling)
+    bound = [plans[mb].bind(*halves[mb]) for mb in range(2)]
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    comp = torch.cuda.current_stream()
+
+    def step():
+        flush.zero_()
+        ev = torch.cuda.Event()
+        ev.record(comp)
+        for mb in range(2):
+            streams[mb].wait_event(ev)
+            plans[mb](bound[mb], stream=streams[mb])
+        for mb in range(2):
+            comp.wait_stream(streams[mb])
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    tot = 0.0
+    for _ in range(steps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(comp)
+        step()
+        e1.record(comp)
+        e1.synchronize()
+        tot += e0.elapsed_time(e1)
+    for pl in plans:
+        rc, word = pl.status()
+        if rc != 0:
+            raise RuntimeError(f"ping-pong plan status {rc} word {word:#x}")
+        pl.close()
+    return tot / steps
 
 
 def run_sweep(args):
@@ -435,8 +519,10 @@ def main():
     counts = to_device_counts(inp)
     flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
     stream = torch.cuda.current_stream()
+    # the slab set is marshalled once, as a serving loop with fixed receive buffers would
+    bound = layer.bind(slabs, counts)
 
-    layer(slabs, counts)
+    layer(bound)
     rc, word = layer.status()
     if rc != 0:
         raise RuntimeError(f"layer status {rc} word {word:#x}")
@@ -447,7 +533,7 @@ def main():
     layer.set_timing(True)
     for _ in range(args.warmup):
         flush.zero_()
-        layer(slabs, counts)
+        layer(bound)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -470,7 +556,7 @@ def main():
                 e0 = torch.cuda.Event(enable_timing=True)
                 e1 = torch.cuda.Event(enable_timing=True)
                 e0.record(stream)
-                layer(slabs, counts)
+                layer(bound)
                 e1.record(stream)
                 e1.synchronize()
                 step_ms.append(e0.elapsed_time(e1))
@@ -478,7 +564,7 @@ def main():
     # stage times: a few further calls with per-kernel events (not part of the timed steps)
     for _ in range(min(args.steps, 5)):
         flush.zero_()
-        layer(slabs, counts)
+        layer(bound)
         torch.cuda.synchronize()
         for k, v in layer.kernel_times().items():
             kt[k].append(v)
@@ -498,7 +584,7 @@ def main():
     # for context: the same call replayed from a CUDA graph (the direct-launch time above
     # stays the reported value)
     graph_ms = None
-    if not args.graph:
+    if not args.graph and not args.quick:
         gms = time_layer(layer, slabs, counts, flush, min(args.steps, 10), 2, graph=True)
         graph_ms = float(np.mean(gms))
         if world > 1:
@@ -512,43 +598,57 @@ def main():
     # end to end through the public API from pinned host memory (uploads, layer and
     # downloads inside the timed region), serial and two-deep pipelined
     layer.set_timing(False)
-    slabs2 = to_device_slabs(inp, y_fill=0.0)
-    counts2 = to_device_counts(inp)
-    e2e_serial_ms, e2e_pipe_ms, h2d, d2h = time_e2e(layer, inp, [slabs, slabs2], [counts, counts2],
-                                                    flush, args.steps, args.warmup)
-    if world > 1:
-        t = torch.tensor([e2e_serial_ms, e2e_pipe_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_serial_ms, e2e_pipe_ms = (float(v) for v in t.tolist())
-    rc, word = layer.status()
-    if rc != 0:
-        raise RuntimeError(f"layer status {rc} word {word:#x} after the end-to-end steps")
+    e2e = None
+    ping_pong = None
+    if not args.quick:
+        slabs2 = to_device_slabs(inp, y_fill=0.0)
+        counts2 = to_device_counts(inp)
+        e2e_serial_ms, e2e_pipe_ms, h2d, d2h = time_e2e(layer, inp, [slabs, slabs2], [counts, counts2],
+                                                        flush, args.steps, args.warmup)
+        del slabs2, counts2
+        if world > 1:
+            t = torch.tensor([e2e_serial_ms, e2e_pipe_ms], device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_serial_ms, e2e_pipe_ms = (float(v) for v in t.tolist())
+        rc, word = layer.status()
+        if rc != 0:
+            raise RuntimeError(f"layer status {rc} word {word:#x} after the end-to-end steps")
+        e2e = {"value": world * T / (e2e_pipe_ms * 1e-3), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": e2e_pipe_ms,
+               "mode": "two-deep pipeline: upload of step i+1 and download of step i-1 on "
+                       "copy streams during step i; L2 flush before each layer call, timed",
+               "serial": {"value": world * T / (e2e_serial_ms * 1e-3), "ms_per_step": e2e_serial_ms}}
+        # k = 2 ping-pong microbatches: every slab split into two halves, each half served
+        # by its own plan over the same weights on its own stream
+        pp_ms = time_ping_pong(inp, dev_w, slabs, flush, args.steps, args.warmup, args.tiling)
+        if world > 1:
+            t = torch.tensor([pp_ms], device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            pp_ms = float(t.item())
+        ping_pong = {"ms_per_step": pp_ms, "tokens_per_s": world * T / (pp_ms * 1e-3),
+                     "mode": "two plans over one weight set, microbatch A = first half of every "
+                             "slab's rows on stream 0, B = the rest on stream 1, both per step; "
+                             "L2 flushed before each step"}
 
     hbm, bf16, bf16_sus, peak_src = measured_peaks()
     fp8_peak = 2.0 * bf16          # measured bf16 burst x nominal fp8/bf16 ratio 2
     mean = {k: float(np.mean(v)) for k, v in kt.items()}
     H, I = inp.shape.hidden, inp.shape.intermediate
-    if tiling == 4:
-        # one persistent launch runs both projections; its time is the W13 stage's
-        dominant, t_dom, flops_k = "fused_w13_w2", mean["gemm13_swiglu"], 6.0 * H * I * R
-    else:
-        dominant = max(("gemm13_swiglu", "gemm2_combine"), key=lambda k: mean[k])
-        t_dom = mean[dominant]
-        flops_k = (4.0 if dominant == "gemm13_swiglu" else 2.0) * H * I * R
+    dominant = max(("gemm13_swiglu", "gemm2_combine"), key=lambda k: mean[k])
+    t_dom = mean[dominant]
+    flops_k = (4.0 if dominant == "gemm13_swiglu" else 2.0) * H * I * R
     achieved = flops_k / (t_dom * 1e-3) / 1e12
-    # stage times as launched: the scan runs inside route_count; the default tiling runs
-    # both projections in one launch
+    # stage times as launched: the scan runs inside route_count
     stage_ms = dict(mean)
     stage_ms["route_count_scan"] = stage_ms.pop("route_count") + stage_ms.pop("route_scan")
-    if tiling == 4:
-        stage_ms["fused_w13_w2"] = stage_ms.pop("gemm13_swiglu") + stage_ms.pop("gemm2_combine")
     t_roof = max(bytes_alg / (hbm * 1e9), flops_alg / (fp8_peak * 1e12))
     layer_ms = tot_ms / args.steps
     bound = "tensor" if flops_alg / (fp8_peak * 1e12) >= bytes_alg / (hbm * 1e9) else "hbm"
 
     if rank == 0:
         cpu = None
-        if not args.no_cpu_baseline and world == 1:
+        if not args.no_cpu_baseline and not args.quick and world == 1:
             cpu = cpu_baseline(inp, args.cpu_sample_tokens)
         line = {
             "metric": METRIC,
@@ -564,12 +664,10 @@ def main():
             "dtype": "fp8_e4m3",
             "data": "synthetic",
             "config": workload_config(wl, inp, rt, world),
-            "kernel_config": {"gemm_tiling": {1: "one CTA per 128x256 tile, W13 and W2 as two launches",
-                                              4: "one CTA per 128x256 tile, W13 and W2 in one persistent launch",
-                                              2: "CTA pairs on 256x256 tiles (cta_group::2)",
-                                              3: "one CTA per 128x256 tile, W13 rows by tile::gather4",
-                                              5: "one CTA per 128x256 tile, W13 on the block-scale MMA path "
-                                                 "(power-of-two scales), W2 as two-launch"}[tiling],
+            "kernel_config": {"gemm_tiling": {1: "one CTA per 128x256 tile, software promotion of "
+                                                 "every 128-wide K block (any fp32 block scales)",
+                                              2: "one CTA per 128x256 tile, W13 on the block-scale MMA path "
+                                                 "(power-of-two scales), W2 software-promoted"}[tiling],
                               "launch": "CUDA graph replay" if args.graph else "direct launches"},
             "roofline": {"bound": "tensor", "kernel": dominant, "achieved": achieved,
                          "peak": fp8_peak, "unit": "TFLOP/s", "frac": achieved / fp8_peak,
@@ -581,13 +679,9 @@ def main():
             "kernel_ms": stage_ms,
             "graph_replay_ms_per_step": graph_ms,
             "routed_rows_per_s": world * args.steps * R / (tot_ms * 1e-3),
-            "e2e": {"value": world * T / (e2e_pipe_ms * 1e-3), "unit": "tokens/s",
-                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "ms_per_step": e2e_pipe_ms,
-                    "mode": "two-deep pipeline: upload of step i+1 and download of step i-1 on "
-                            "copy streams during step i; L2 flush before each layer call, timed",
-                    "serial": {"value": world * T / (e2e_serial_ms * 1e-3), "ms_per_step": e2e_serial_ms}},
-            "gpu_launches": (kernels_per_layer() + {4: -1, 5: 1}.get(tiling, 0)) * args.steps,
+            "e2e": e2e,
+            "ping_pong_k2": ping_pong,
+            "gpu_launches": kernels_per_layer(layer) * args.steps,
             "clocks": clk.summary(),
             "cpu_baseline": cpu,
         }

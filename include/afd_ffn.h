@@ -71,7 +71,7 @@ typedef enum {
 #define AFD_STATUS_BAD_ROUTING 0x1 /* id outside [0, E_g) and != -1, or repeated in a token */
 #define AFD_STATUS_TIMEOUT 0x2     /* a bounded device wait expired; outputs are invalid */
 #define AFD_STATUS_BAD_COUNT 0x4   /* some counts[m] < 0 or > slab_capacity; clamped */
-#define AFD_STATUS_BAD_SCALE 0x8   /* tiling 5: an activation block scale of this call is not a
+#define AFD_STATUS_BAD_SCALE 0x8   /* tiling 2: an activation block scale of this call is not a
                                       positive normal power of two; outputs are invalid */
 
 /* Limits. */
@@ -82,10 +82,9 @@ typedef enum {
 
 /* Timed stages of one layer call, in launch order (for afd_ffn_get_kernel_times). One
  * kernel per stage, except that the routing scan runs in the last block of the route
- * count kernel: AFD_KERNEL_ROUTE_COUNT covers both and AFD_KERNEL_ROUTE_SCAN reads as
- * zero. The gather stage copies the routed FP8 rows and their scales into expert order;
- * with tiling 3 it moves only the scales (the W13 kernel then fetches the rows from the
- * slabs itself). */
+ * count kernel (AFD_KERNEL_ROUTE_COUNT covers both and AFD_KERNEL_ROUTE_SCAN reads as
+ * zero) and that with a shared expert the down projection writes the slab rows itself
+ * (AFD_KERNEL_FINALIZE reads as zero). The gather stage copies the routed FP8 rows and their scales into expert order. */
 #define AFD_KERNEL_ROUTE_COUNT 0
 #define AFD_KERNEL_ROUTE_SCAN 1
 #define AFD_KERNEL_ROUTE_SCATTER 2
@@ -219,19 +218,11 @@ AFD_API afd_status_t afd_ffn_get_kernel_times(afd_ffn_plan_t plan, float* ms);
 
 /*
  * Tiling of the two grouped GEMMs, chosen on the host for the following calls.
- * 0 (default) or 1: one CTA per 128-row x 256-column tile, A rows from the gather stage's
- * expert-ordered copy; W13 and W2 are two launches.
- * 2: CTA pairs on 256-row tiles (cta_group::2 MMAs, less operand traffic per MMA, but a
- *    per-K-block handshake between the two SMs that measured about 2x slower).
- * 3: as 1, but the W13 kernel fetches its A rows straight from the slabs with TMA
- *    tile::gather4 (no row copy; 32 four-row requests per A tile, measured about 2.7x
- *    slower for W13 on a 4096-token DeepSeek-V3 share).
- * 4: as 1, but W13 and W2 run in one persistent launch: every CTA walks its W13 tiles and
- *    then its W2 tiles; a W2 tile waits (bounded) on a per-m-tile counter that the W13
- *    epilogues of its m-tile release. Measured slower than two launches on the 4096-token
- *    DeepSeek-V3 share (1582 against 1446 us) although each half alone runs at its
- *    two-launch speed.
- * 5: as 1, but W13 runs on the tensor core's block-scale path (kind::mxf8f6f4 with UE8M0
+ * 0 (default) or 1: one CTA per 128-row x 256-column tile; every 128-wide K block is a
+ *    separate tensor-core partial product that the epilogue scales by (activation block
+ *    scale x weight block scale) and accumulates in fp32 registers, so any positive fp32
+ *    block scales are exact.
+ * 2: as 1, but W13 runs on the tensor core's block-scale path (kind::mxf8f6f4 with UE8M0
  *    factors): TMEM accumulates a tile's whole K loop and the epilogue runs once per
  *    tile. Only for inputs whose activation and W13 block scales are all positive normal
  *    powers of two (each is then exactly its UE8M0 factor). The first selection on a plan
@@ -243,13 +234,13 @@ AFD_API afd_status_t afd_ffn_get_kernel_times(afd_ffn_plan_t plan, float* ms);
  *    images), which checks that call's activation scales: any other scale sets
  *    AFD_STATUS_BAD_SCALE, on every such call, and afd_ffn_get_status then returns
  *    AFD_ERR_INVALID_ARGUMENT.
- * Results are the same within rounding; tilings 2, 3, 4 and 5 exist for tests and
- * measurements. afd_ffn_kernels_per_layer counts the default tiling's launches (tiling 4
- * makes one fewer, tiling 5 one more). Returns AFD_ERR_INVALID_ARGUMENT outside 0..5.
+ * Results are the same within rounding. Returns AFD_ERR_INVALID_ARGUMENT outside 0..2.
  */
+#define AFD_TILING_DEFAULT 1
+#define AFD_TILING_BLOCK_SCALE 2
 AFD_API afd_status_t afd_ffn_set_tiling(afd_ffn_plan_t plan, int32_t tiling);
 
-/* Synchronise `stream` and report the tiling (1 to 5) the last layer call used. */
+/* Synchronise `stream` and report the tiling (1 or 2) the last layer call used. */
 AFD_API afd_status_t afd_ffn_get_tiling(afd_ffn_plan_t plan, afd_stream_t stream, int32_t* tiling);
 
 /*
@@ -303,8 +294,10 @@ AFD_API afd_status_t afd_ffn_route_noalloc(const afd_ffn_config_t* cfg, const af
                                            float* d_row_weight, int32_t* d_pos, int32_t* d_status,
                                            afd_stream_t stream);
 
-/* Number of this library's kernel launches one afd_ffn_layer call makes. */
-AFD_API int32_t afd_ffn_kernels_per_layer(void);
+/* Number of this library's kernel launches one afd_ffn_layer call of this plan makes with
+ * its current tiling: 5 with a shared expert, 6 without (a separate finalisation writes the
+ * slab rows), one more with tiling 2. -1 for NULL. */
+AFD_API int32_t afd_ffn_kernels_per_layer(afd_ffn_plan_t plan);
 
 /* Human-readable name of a status code. */
 AFD_API const char* afd_status_string(afd_status_t s);

@@ -87,43 +87,18 @@ def route_inputs(inp) -> Routing:
                  [s.topk_weights for s in inp.slabs])
 
 
-def ffn_layer(inp, tokens: Optional[Sequence[int]] = None, routing: Optional[Routing] = None,
-              keep_intermediates: bool = False):
-    """Grouped form: rows grouped by expert, one dense product per expert.
+def _wanted_rows(rt: Routing, e: int, want: np.ndarray) -> np.ndarray:
+    r0, r1 = int(rt.offsets[e]), int(rt.offsets[e + 1])
+    rows = np.arange(r0, r1)
+    return rows[want[rt.row_token[rows]]]
 
-    Returns a dict with 'out' (float64 [n, H], before bf16 rounding), 'out_bf16'
-    (float64 values of the bf16 result), 'tokens' (the global token ids of the rows of
-    'out'), 'routing', and optionally per-row 'h_codes' / 'h_scales' / 'Y'.
-    """
-    sh = inp.shape
-    H, I, El, S = sh.hidden, sh.intermediate, sh.num_local_experts, sh.has_shared_expert
-    rt = routing if routing is not None else route_inputs(inp)
-    T = rt.num_tokens
-    toks = np.arange(T) if tokens is None else np.asarray(tokens, np.int64)
-    want = np.zeros(T, bool)
-    want[toks] = True
-    xc, xs = gather_tokens(inp, rt)
-    R = rt.num_rows
-    Y = np.zeros((R, H), np.float64)
-    h_codes = np.zeros((R, I), np.uint8) if keep_intermediates else None
-    h_scales = np.zeros((R, I // QB), np.float32) if keep_intermediates else None
-    for e in range(El + S):
-        r0, r1 = int(rt.offsets[e]), int(rt.offsets[e + 1])
-        rows = np.arange(r0, r1)
-        rows = rows[want[rt.row_token[rows]]]
-        if rows.size == 0:
-            continue
-        x = dequant_rows(xc[rt.row_token[rows]], xs[rt.row_token[rows]])
-        w13 = dequant_weight(inp.w13[e], inp.w13_scale[e])
-        w2 = dequant_weight(inp.w2[e], inp.w2_scale[e])
-        y, q, s = expert_forward(x, w13, w2, I)
-        Y[rows] = y
-        if keep_intermediates:
-            h_codes[rows], h_scales[rows] = q, s
-    out = np.zeros((toks.size, H), np.float64)
-    K = sh.top_k
+
+def _combine(rt: Routing, Y: np.ndarray, toks: np.ndarray, K: int, El: int, S: int) -> np.ndarray:
+    """out[g] = sum over local slots k (ascending) of w[g,k] * Y[pos[g,k]] + S * Y[shared
+    row of g], in float64."""
+    out = np.zeros((toks.size, Y.shape[1]), np.float64)
     for i, g in enumerate(toks):
-        acc = np.zeros(H, np.float64)
+        acc = np.zeros(Y.shape[1], np.float64)
         for k in range(K):
             r = rt.pos[g * K + k]
             if r >= 0:
@@ -131,10 +106,76 @@ def ffn_layer(inp, tokens: Optional[Sequence[int]] = None, routing: Optional[Rou
         if S:
             acc += Y[rt.offsets[El] + g]
         out[i] = acc
+    return out
+
+
+def _want(rt: Routing, tokens) -> tuple:
+    T = rt.num_tokens
+    toks = np.arange(T) if tokens is None else np.asarray(tokens, np.int64)
+    want = np.zeros(T, bool)
+    want[toks] = True
+    return toks, want
+
+
+def ffn_layer(inp, tokens: Optional[Sequence[int]] = None, routing: Optional[Routing] = None,
+              keep_intermediates: bool = False):
+    """Grouped form: rows grouped by expert, one dense product per expert.
+
+    Returns a dict with 'out' (float64 [n, H], before bf16 rounding), 'out_bf16'
+    (float64 values of the bf16 result), 'tokens' (the global token ids of the rows of
+    'out'), 'routing', and optionally per-row 'h32' (the float32 intermediate the
+    quantisation decision is taken on), 'h_codes' / 'h_scales' and 'Y'. Rows of tokens
+    outside `tokens` are left zero.
+    """
+    sh = inp.shape
+    H, I, El, S = sh.hidden, sh.intermediate, sh.num_local_experts, sh.has_shared_expert
+    rt = routing if routing is not None else route_inputs(inp)
+    toks, want = _want(rt, tokens)
+    xc, xs = gather_tokens(inp, rt)
+    R = rt.num_rows
+    Y = np.zeros((R, H), np.float64)
+    if keep_intermediates:
+        h32 = np.zeros((R, I), np.float32)
+        h_codes = np.zeros((R, I), np.uint8)
+        h_scales = np.zeros((R, I // QB), np.float32)
+    for e in range(El + S):
+        rows = _wanted_rows(rt, e, want)
+        if rows.size == 0:
+            continue
+        x = dequant_rows(xc[rt.row_token[rows]], xs[rt.row_token[rows]])
+        w13 = dequant_weight(inp.w13[e], inp.w13_scale[e])
+        w2 = dequant_weight(inp.w2[e], inp.w2_scale[e])
+        G = x @ w13.T
+        h = swiglu(G[:, :I], G[:, I:])
+        q, s, hq = requant_rows(h)
+        Y[rows] = hq @ w2.T
+        if keep_intermediates:
+            h32[rows], h_codes[rows], h_scales[rows] = h.astype(np.float32), q, s
+    out = _combine(rt, Y, toks, sh.top_k, El, S)
     res = {"out": out, "out_bf16": bf16_round(out), "tokens": toks, "routing": rt}
     if keep_intermediates:
-        res.update(h_codes=h_codes, h_scales=h_scales, Y=Y)
+        res.update(h32=h32, h_codes=h_codes, h_scales=h_scales, Y=Y)
     return res
+
+
+def down_and_combine(inp, routing: Routing, h_codes: np.ndarray, h_scales: np.ndarray,
+                     tokens: Optional[Sequence[int]] = None) -> np.ndarray:
+    """The layer's second half from a given intermediate: for every row of the wanted
+    tokens, Y = dequant(h_codes, h_scales) . W2_f^T of its expert, then the combine.
+    With the codes and scales ffn_layer computes itself this returns its 'out' exactly.
+    Returns float64 [n, H] before bf16 rounding."""
+    sh = inp.shape
+    H, El, S = sh.hidden, sh.num_local_experts, sh.has_shared_expert
+    rt = routing
+    toks, want = _want(rt, tokens)
+    Y = np.zeros((rt.num_rows, H), np.float64)
+    for e in range(El + S):
+        rows = _wanted_rows(rt, e, want)
+        if rows.size == 0:
+            continue
+        w2 = dequant_weight(inp.w2[e], inp.w2_scale[e])
+        Y[rows] = dequant_rows(h_codes[rows], h_scales[rows]) @ w2.T
+    return _combine(rt, Y, toks, sh.top_k, El, S)
 
 
 def ffn_layer_bruteforce(inp) -> np.ndarray:

@@ -13,7 +13,7 @@ import pytest
 import workloads as W
 from oracle import ffn as offn
 from oracle import fp8 as ofp8
-from tests.helpers import TOL_ROW_RMS, compare_outputs, run_cuda_layer
+from tests.helpers import TOL_ROW_RMS, compare_layer, reconcile_codes, run_cuda_layer
 
 pytestmark = pytest.mark.gpu
 
@@ -31,13 +31,21 @@ def test_two_expert_shards_sum_to_the_full_layer(counts, cap, zipf):
     full = W.make_custom_inputs(W.LayerShape(H, I, Eg, 0, Eg, 1, K), counts, cap, seed=41, zipf_s=zipf)
     a = _shard(full, W.LayerShape(H, I, Eg, 0, 8, 1, K), 0, 8, True)
     b = _shard(full, W.LayerShape(H, I, Eg, 8, 8, 0, K), 8, 16, False)
-    ref = offn.ffn_layer(full)["out"]
-    parts = []
+    parts, refs = [], []
     for shard in (a, b):
         res = run_cuda_layer(shard)
         assert res["status_rc"] == 0
-        compare_outputs(res["outs"][0], offn.ffn_layer(shard)["out"])
+        compare_layer(res, shard)
         parts.append(ofp8.bf16_from_bits(res["outs"][0]))
+        # the shard's oracle with the GPU's midpoint decisions (if any) taken over
+        o = offn.ffn_layer(shard, keep_intermediates=True)
+        rows = np.arange(o["routing"].num_rows)
+        codes, _ = reconcile_codes(res["h_codes"], res["h_scales"], o["h32"], o["h_codes"],
+                                   o["h_scales"], rows)
+        refs.append(offn.down_and_combine(shard, o["routing"], codes, o["h_scales"]))
+    # the full layer is the sum of the shards' partial sums (the oracle's own pin of this is
+    # in the CPU tests); the GPU's two bf16 partials must add up to it
+    ref = refs[0] + refs[1]
     total = parts[0] + parts[1]
     rms = np.sqrt((ref ** 2).mean(axis=1))
     err = np.abs(total - ref).max(axis=1)

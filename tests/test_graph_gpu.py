@@ -12,7 +12,7 @@ import torch
 
 import workloads as W
 from oracle import ffn as offn
-from tests.helpers import compare_outputs, compare_routing
+from tests.helpers import compare_layer
 
 pytestmark = pytest.mark.gpu
 
@@ -64,9 +64,9 @@ def test_layer_replays_from_a_cuda_graph_with_new_inputs():
         torch.cuda.synchronize()
         g.replay()
         torch.cuda.synchronize()
-        ref = offn.ffn_layer(inp)
-        compare_routing(layer.routing(), ref["routing"])
-        compare_outputs(gather_outputs(inp, slabs), ref["out"])
+        codes, scales = layer.intermediate()
+        compare_layer({"outs": [gather_outputs(inp, slabs)], "routing": layer.routing(),
+                       "h_codes": codes, "h_scales": scales}, inp)
     rc, word = layer.status()
     assert rc == 0, word
     del g

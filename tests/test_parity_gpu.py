@@ -11,17 +11,17 @@ import pytest
 
 import workloads as W
 from oracle import ffn as offn
-from tests.helpers import compare_outputs, compare_routing, run_cuda_layer, structural_tokens
+from tests.helpers import compare_layer, compare_outputs, run_cuda_layer, structural_tokens
 
 pytestmark = pytest.mark.gpu
 
 
 def _full_check(inp, calls=1, tiling=0):
+    """Every output row of every call against the oracle (tests.helpers.compare_layer)."""
     res = run_cuda_layer(inp, calls=calls, tiling=tiling)
-    ref = offn.ffn_layer(inp)
-    compare_routing(res["routing"], ref["routing"])
-    worst = [compare_outputs(o, ref["out"]) for o in res["outs"]]
-    return res, ref, worst
+    rt = offn.route_inputs(inp)
+    worst, flips = compare_layer(res, inp, routing=rt)
+    return res, rt, worst
 
 
 def test_tiny_config():
@@ -42,36 +42,49 @@ def test_random_shapes_several_tiles(seed, shape, counts, cap, zipf):
     assert res["status_rc"] == 0
 
 
-@pytest.mark.parametrize("tiling", [1, 2, 3, 4])
 @pytest.mark.parametrize("seed,shape,counts,cap", [
-    # experts of a few hundred rows: pair tiles whose second CTA is partly or fully empty
+    # experts of a few hundred rows with ragged last tiles, an empty slab, a single token
     (21, W.LayerShape(512, 256, 4, 0, 4, 1, 2), [300, 217, 0, 65], 300),
     (22, W.LayerShape(768, 384, 6, 0, 6, 0, 3), [511, 2], 511),
     (23, W.LayerShape(1024, 256, 16, 4, 6, 1, 4), [1, 0, 130], 130),
 ])
-def test_both_tilings(tiling, seed, shape, counts, cap):
+def test_ragged_tiles_two_calls(seed, shape, counts, cap):
     inp = W.make_custom_inputs(shape, counts, cap, seed=seed, zipf_s=1.0)
-    res, _, _ = _full_check(inp, calls=2, tiling=tiling)
-    assert res["tiling"] == tiling
+    res, _, _ = _full_check(inp, calls=2)
+    assert res["tiling"] == 1
+    assert res["status_rc"] == 0
+
+
+# Small batches: when a projection's tiles fill at most half of the GPU, each tile's K
+# blocks are shared out among CTAs (split-K). H = I = 1024 gives 8 K blocks per tile, so
+# both projections split in two; with a shared expert only W13 splits. Three calls check
+# that the split workspace and its counters are clear again after every call.
+@pytest.mark.parametrize("shape,counts,cap", [
+    (W.LayerShape(1024, 1024, 8, 0, 8, 0, 2), [3], 3),
+    (W.LayerShape(1024, 1024, 8, 0, 8, 0, 2), [1, 0, 16], 16),
+    (W.LayerShape(1024, 1024, 16, 4, 8, 1, 4), [5, 2], 5),
+    (W.LayerShape(2048, 1024, 8, 0, 6, 1, 3), [1], 1),
+])
+def test_split_k_small_batches(shape, counts, cap):
+    inp = W.make_custom_inputs(shape, counts, cap, seed=51, zipf_s=1.0)
+    res, _, _ = _full_check(inp, calls=3)
     assert res["status_rc"] == 0
 
 
 # The ABI's limits in one layer: 1024 groups (1023 local experts + shared), top-K 32 and
-# 128 slabs of two tokens each; every tiling (the slab-gather tiling then carries 128
-# per-slab tensor maps).
+# 128 slabs of two tokens each.
 _LIMITS_SHAPE = W.LayerShape(256, 128, 1024, 0, 1023, 1, 32)
 
 
-@pytest.mark.parametrize("tiling", [1, 2, 3, 4])
-def test_limits_groups_topk_slabs(tiling):
+def test_limits_groups_topk_slabs():
     inp = W.make_custom_inputs(_LIMITS_SHAPE, [2] * 128, 2, seed=31)
-    res, ref, _ = _full_check(inp, calls=1, tiling=tiling)
-    assert res["tiling"] == tiling and res["status_rc"] == 0
+    res, ref, _ = _full_check(inp, calls=1)
+    assert res["status_rc"] == 0
     # id 1023 is not held here, so a token that picked it has 31 local rows + shared
-    assert 256 * 31 < ref["routing"].num_rows <= 256 * 33
+    assert 256 * 31 < ref.num_rows <= 256 * 33
 
 
-# Tiling 5: W13 on the block-scale MMA path, for power-of-two block scales. The oracle is
+# Tiling 2: W13 on the block-scale MMA path, for power-of-two block scales. The oracle is
 # the same; only the inputs' scales are rounded up to powers of two.
 @pytest.mark.parametrize("seed,shape,counts,cap", [
     (21, W.LayerShape(512, 256, 4, 0, 4, 1, 2), [300, 217, 0, 65], 300),
@@ -81,15 +94,15 @@ def test_limits_groups_topk_slabs(tiling):
 ])
 def test_block_scale_tiling(seed, shape, counts, cap):
     inp = W.make_custom_inputs(shape, counts, cap, seed=seed, zipf_s=1.0, pow2_scales=True)
-    res, _, _ = _full_check(inp, calls=2, tiling=5)
-    assert res["tiling"] == 5
+    res, _, _ = _full_check(inp, calls=2, tiling=2)
+    assert res["tiling"] == 2
     assert res["status_rc"] == 0
 
 
 def test_block_scale_tiling_limits():
     inp = W.make_custom_inputs(_LIMITS_SHAPE, [2] * 128, 2, seed=31, pow2_scales=True)
-    res, _, _ = _full_check(inp, calls=1, tiling=5)
-    assert res["tiling"] == 5 and res["status_rc"] == 0
+    res, _, _ = _full_check(inp, calls=1, tiling=2)
+    assert res["tiling"] == 2 and res["status_rc"] == 0
 
 
 def test_block_scale_tiling_refuses_other_weight_scales():
@@ -100,15 +113,15 @@ def test_block_scale_tiling_refuses_other_weight_scales():
     inp = W.make_inputs(W.CONFIGS["tiny"])
     layer = FfnLayer(inp.shape, len(inp.slabs), inp.capacity, *to_device_weights(inp))
     with pytest.raises(AfdError) as e:
-        layer.set_tiling(5)
+        layer.set_tiling(2)
     assert e.value.code == 1
     res = run_cuda_layer(inp, layer=layer)
     assert res["status_rc"] == 0 and res["tiling"] == 1
-    compare_outputs(res["outs"][0], offn.ffn_layer(inp)["out"])
+    compare_layer(res, inp)
 
 
 def test_block_scale_tiling_flags_activation_scales_on_every_call():
-    """Power-of-two W13 scales but amax/448 activation scales: every tiling-5 call sets
+    """Power-of-two W13 scales but amax/448 activation scales: every tiling-2 call sets
     BAD_SCALE, also after afd_ffn_get_status has cleared the word."""
     from attention_ffn_disaggregated_b200 import FfnLayer
     from attention_ffn_disaggregated_b200.device import (to_device_counts, to_device_slabs,
@@ -118,7 +131,7 @@ def test_block_scale_tiling_flags_activation_scales_on_every_call():
     wts = W.make_custom_inputs(sh, [40], 40, seed=41, pow2_scales=True)
     acts = W.make_custom_inputs(sh, [40], 40, seed=41)
     layer = FfnLayer(sh, 1, 40, *to_device_weights(wts))
-    layer.set_tiling(5)
+    layer.set_tiling(2)
     slabs, counts = to_device_slabs(acts), to_device_counts(acts)
     for _ in range(2):
         layer(slabs, counts)
@@ -127,10 +140,10 @@ def test_block_scale_tiling_flags_activation_scales_on_every_call():
 
 
 def test_repeated_calls_self_clean():
-    """The combine accumulators are cleared by the last contributor: call twice, same result."""
+    """The combine accumulators are zero again after every call: three calls, each correct."""
     inp = W.make_custom_inputs(W.LayerShape(512, 256, 12, 2, 8, 1, 4), [200, 90], 200, seed=7)
-    res, ref, worst = _full_check(inp, calls=3)
-    assert len(worst) == 3
+    res, _, _ = _full_check(inp, calls=3)
+    assert len(res["outs"]) == 3
 
 
 def test_empty_batch_and_empty_slabs():
@@ -175,8 +188,11 @@ def test_count_above_capacity_is_clamped_and_flagged():
     layer(slabs, torch.tensor([9, 4], dtype=torch.int32, device="cuda"))
     rc, word = layer.status()
     assert word & 0x4 and rc == 5
-    ref = offn.ffn_layer(inp)              # counts clamp to capacity: same as [4, 4]
-    compare_outputs(gather_outputs(inp, slabs), ref["out"])
+    # counts clamp to capacity: the same layer as counts [4, 4]
+    codes, scales = layer.intermediate()
+    res = {"outs": [gather_outputs(inp, slabs)], "routing": layer.routing(), "h_codes": codes,
+           "h_scales": scales}
+    compare_layer(res, inp)
 
 
 def test_single_token_single_slab():
@@ -184,17 +200,18 @@ def test_single_token_single_slab():
     _full_check(inp)
 
 
-def test_intermediate_codes_match_oracle_mostly():
-    """Diagnostic on h: FP8 codes equal to the oracle's except rare rounding-boundary flips."""
+def test_intermediate_codes_match_oracle():
+    """The intermediate itself: every FP8 code equal to the oracle's, or the adjacent value
+    across a rounding midpoint that the oracle's h/scale lies within float32 noise of;
+    block scales within 1e-4 relative."""
+    from tests.helpers import reconcile_codes
     inp = W.make_custom_inputs(W.LayerShape(512, 256, 8, 0, 8, 0, 2), [160, 100], 160, seed=14)
     res = run_cuda_layer(inp)
     ref = offn.ffn_layer(inp, keep_intermediates=True)
-    codes, scales = res["layer"].intermediate()
     R = ref["routing"].num_rows
-    assert codes.shape == (R, 256)
-    same = codes == ref["h_codes"]
-    assert same.mean() > 0.995, same.mean()
-    np.testing.assert_allclose(scales, ref["h_scales"], rtol=1e-4)
+    assert res["h_codes"].shape == (R, 256)
+    reconcile_codes(res["h_codes"], res["h_scales"], ref["h32"], ref["h_codes"], ref["h_scales"],
+                    np.arange(R))
 
 
 def test_timeout_injection_reports_status_and_recovers():
@@ -210,27 +227,28 @@ def test_timeout_injection_reports_status_and_recovers():
     layer.set_wait_limit(1_000_000_000)
     again = run_cuda_layer(inp, layer=layer)
     assert again["status_rc"] == 0
-    compare_outputs(again["outs"][0], offn.ffn_layer(inp)["out"])
+    compare_layer(again, inp)
 
 
 # ------------------------------------------------------------------ full-size workloads
 
 def _full_size_check(inp, n_total=None, tiling=0):
-    """Routing bit-exact on every token; outputs against the oracle on every token, or on
-    the structural selection of tests.helpers.structural_tokens when n_total is given."""
+    """Routing bit-exact on every token; intermediate and outputs against the oracle on
+    every token, or on the structural selection of tests.helpers.structural_tokens when
+    n_total is given."""
     res = run_cuda_layer(inp, tiling=tiling)
     assert res["status_rc"] == 0, res["status_word"]
     ort = offn.route_inputs(inp)
-    compare_routing(res["routing"], ort)
     toks = (None if n_total is None else
             structural_tokens(ort, inp.counts, n_total, inp.shape.num_local_experts))
-    ref = offn.ffn_layer(inp, tokens=toks, routing=ort)
-    return compare_outputs(res["outs"][0], ref["out"], tokens=toks), res
+    worst, flips = compare_layer(res, inp, tokens=toks, routing=ort)
+    print(f"worst row error {worst:.4f} x RMS, {flips} midpoint codes")
+    return worst, res
 
 
 @pytest.mark.parametrize("name,tiling", [("qwen3_235b_t2048", 0), ("deepseek_v3_share_t4096", 0),
                                          ("qwen3_235b_spec_q4_t8192", 0),
-                                         ("deepseek_v3_share_t4096_pow2", 5)])
+                                         ("deepseek_v3_share_t4096_pow2", 2)])
 def test_full_size_every_token(name, tiling):
     """The three full-size workloads (and the block-scale tiling on the power-of-two twin of
     the DeepSeek-V3 share): every output row against the oracle."""
