@@ -26,20 +26,16 @@
 
 using namespace afd;
 
-// Tile order of the down projection: 0 = m-tile major, 1 = column-tile major (every
-// m-tile of a 256-column slice before the next slice).
+// Tile order of the down projection: column-tile major (every m-tile of a 256-column
+// slice before the next slice). Each slice's weight rows are then read from DRAM once,
+// while the intermediate (re-read by every slice, evict-last) and the slice's live
+// accumulators stay in L2; in m-tile-major order the 117 MB of accumulators crowd the
+// weights out of L2 between an expert's m-tiles (3.8x the algorithmic DRAM traffic on the
+// DeepSeek-V3 share) at the same kernel time.
 #ifndef AFD_W2_SLICE_FIRST
-#define AFD_W2_SLICE_FIRST 0
-#endif
-// With a shared expert the down projection's shared tiles finish the combine (1); 0 keeps
-// the separate finalisation kernel for every layer.
-#ifndef AFD_FUSE_COMBINE
-#define AFD_FUSE_COMBINE 1
+#define AFD_W2_SLICE_FIRST 1
 #endif
 
-namespace {
-bool fused_combine(const afd_ffn_config_t& c) { return AFD_FUSE_COMBINE && c.has_shared_expert; }
-}  // namespace
 
 namespace {
 
@@ -74,7 +70,6 @@ struct afd_ffn_plan_s {
   int32_t *slab_base, *info, *chunk_hist, *chunk_off, *group_count, *group_off, *mtile_off;
   int tiling = 0;  // 0 = default (1); 2 = block-scale W13
   int32_t *tok_mt, *tok_need, *pos, *row_token, *row_k;
-  int32_t *blk_need = nullptr, *blk_cnt = nullptr;   // fused combine (shared expert only)
   float* g_ws;        // split-K W13: fp32 sums [g_rows][2I], zero between calls
   int g_rows = 0;
   int* g_cnt;         // split-K W13: per (tile, quadrant) counters [num_sms][4]
@@ -110,11 +105,11 @@ const char* afd_status_string(afd_status_t s) {
   return "unknown";
 }
 
-// route count (+ scan), scatter, gather, W13, W2 and, without a shared expert, the
-// finalisation; the block-scale tiling adds the activation factor images
+// route count (+ scan), scatter, gather, W13, W2, finalisation; the block-scale tiling
+// adds the activation factor images
 int32_t afd_ffn_kernels_per_layer(afd_ffn_plan_t P) {
   if (!P) return -1;
-  return 5 + (fused_combine(P->cfg) ? 0 : 1) + (P->tiling == 2 ? 1 : 0);
+  return 6 + (P->tiling == 2 ? 1 : 0);
 }
 
 afd_status_t afd_ffn_check_config(const afd_ffn_config_t* c) {
@@ -131,6 +126,8 @@ afd_status_t afd_ffn_check_config(const afd_ffn_config_t* c) {
   if (c->num_slabs < 1 || c->slab_capacity < 1) return AFD_ERR_INVALID_ARGUMENT;
   // supported limits
   if (c->hidden % 256) return AFD_ERR_UNSUPPORTED;   // W2 output tiles are 256 columns
+  if (c->hidden > AFD_QBLOCK * AFD_MAX_QBLOCKS || c->intermediate > AFD_QBLOCK * AFD_MAX_QBLOCKS)
+    return AFD_ERR_UNSUPPORTED;                      // K blocks held in the GEMMs' scale ring
   if (c->top_k > AFD_MAX_TOP_K) return AFD_ERR_UNSUPPORTED;
   if (c->num_slabs > AFD_MAX_SLABS) return AFD_ERR_UNSUPPORTED;
   if (c->num_local_experts + c->has_shared_expert > AFD_MAX_GROUPS) return AFD_ERR_UNSUPPORTED;
@@ -236,9 +233,6 @@ afd_status_t afd_ffn_plan(const afd_ffn_config_t* cfg, const afd_ffn_weights_t* 
   const size_t o_mtile_off = take(sizeof(int32_t) * (P->G + 1), 16);
   const size_t o_tok_mt = take(sizeof(int32_t) * P->Tmax, 16);
   const size_t o_tok_need = take(sizeof(int32_t) * P->Tmax, 16);
-  const size_t n_blk = static_cast<size_t>(2) * P->num_chunks;   // 128-token blocks, rounded up
-  const size_t o_blk_need = take(S ? sizeof(int32_t) * n_blk : 0, 16);
-  const size_t o_blk_cnt = take(S ? sizeof(int32_t) * n_blk * (H / 256) : 0, 16);
   const size_t o_pos = take(sizeof(int32_t) * static_cast<size_t>(P->Tmax) * K, 16);
   const size_t o_row_token = take(sizeof(int32_t) * P->rpad, 16);
   const size_t o_row_k = take(sizeof(int32_t) * P->rpad, 16);
@@ -278,10 +272,6 @@ afd_status_t afd_ffn_plan(const afd_ffn_config_t* cfg, const afd_ffn_weights_t* 
   P->mtile_off = reinterpret_cast<int32_t*>(b + o_mtile_off);
   P->tok_mt = reinterpret_cast<int32_t*>(b + o_tok_mt);
   P->tok_need = reinterpret_cast<int32_t*>(b + o_tok_need);
-  if (S) {
-    P->blk_need = reinterpret_cast<int32_t*>(b + o_blk_need);
-    P->blk_cnt = reinterpret_cast<int32_t*>(b + o_blk_cnt);
-  }
   P->pos = reinterpret_cast<int32_t*>(b + o_pos);
   P->row_token = reinterpret_cast<int32_t*>(b + o_row_token);
   P->row_k = reinterpret_cast<int32_t*>(b + o_row_k);
@@ -382,9 +372,6 @@ static void fill_route_params(afd_ffn_plan_t P, const int32_t* d_counts, RoutePa
   rp.tiling = P->tiling;
   rp.tok_mt = P->tok_mt;
   rp.tok_need = P->tok_need;
-  rp.blk_need = fused_combine(c) ? P->blk_need : nullptr;
-  rp.blk_cnt = fused_combine(c) ? P->blk_cnt : nullptr;
-  rp.n_ctiles = c.hidden / 256;
   rp.pos = P->pos;
   rp.row_token = P->row_token;
   rp.row_k = P->row_k;
@@ -429,11 +416,7 @@ static void fill_gemm_params(afd_ffn_plan_t P, int epi, GemmParams& gp) {
     gp.row_w = P->row_w;
     gp.acc = P->acc;
     gp.slice_first = P->w2_slice_first;
-    gp.fuse_final = fused_combine(c);
-    gp.split_ok = !fused_combine(c);
-    gp.tok_mt = P->tok_mt;
-    gp.blk_need = P->blk_need;
-    gp.blk_cnt = P->blk_cnt;
+    gp.split_ok = 0;
   }
 }
 
@@ -492,15 +475,13 @@ afd_status_t afd_ffn_layer(afd_ffn_plan_t P, const afd_slab_t* slabs, const int3
                                                                   MxArgs{P->mx_sfa, P->mx_sfb});
   } else {
     grouped_gemm_kernel<EPI_SWIGLU><<<grid, kGemmThreads, gemm_smem_bytes<EPI_SWIGLU>(), stream>>>(
-        g13, P->tm_a13, P->tm_w13, ytab);
+        g13, P->tm_a13, P->tm_w13);
   }
   if (tm) cudaEventRecord(P->ev[5], stream);
   grouped_gemm_kernel<EPI_COMBINE><<<grid, kGemmThreads, gemm_smem_bytes<EPI_COMBINE>(), stream>>>(
-      g2, P->tm_a2, P->tm_w2, ytab);
+      g2, P->tm_a2, P->tm_w2);
   if (tm) cudaEventRecord(P->ev[6], stream);
-  // with a shared expert the down projection's shared tiles write the slab rows themselves
-  if (!fused_combine(c))
-    combine_finalize_kernel<<<P->num_sms * 4, 256, 0, stream>>>(P->info, P->tok_mt, P->acc, c.hidden, ytab);
+  combine_finalize_kernel<<<P->num_sms * 4, 256, 0, stream>>>(P->info, P->tok_mt, P->acc, c.hidden, ytab);
   if (tm) cudaEventRecord(P->ev[7], stream);
   P->ev_valid = tm;
   if (cudaGetLastError() != cudaSuccess) return AFD_ERR_CUDA;

@@ -11,8 +11,8 @@
 // inputs whose scales are all powers of two).
 //
 // Warp roles (384 threads): warp 0 issues TMA loads, warp 1 owns TMEM and issues MMAs,
-// warps 2..3 idle, warps 4..11 are the epilogue (two per TMEM lane quadrant, splitting
-// the columns).
+// warps 2..3 load the weight-block scales of the CTA's next tile into a two-slot ring,
+// warps 4..11 are the epilogue (two per TMEM lane quadrant, splitting the columns).
 //
 // Epilogues:
 //   SWIGLU   (W13) columns are [gate 128 | up 128] of intermediate block nt; h = silu(g)*u
@@ -21,14 +21,8 @@
 //            accumulator by the bulk-copy engine (cp.reduce.async.bulk ... .add.f32: one
 //            512-byte row segment per operation, staged through shared memory), so the
 //            epilogue warps hand the reductions off and return to the next tile's partial
-//            products. With a shared expert (one row per token, in token order, the last
-//            group) the shared expert's tiles are exactly 128-token blocks and come last in
-//            every CTA's tile order: each routed tile, once its reductions are performed,
-//            adds its rows to a counter per (token block, column tile); the shared tile of
-//            that block waits (bounded) until the counter reaches the block's routed-row
-//            count, adds its own rows to the accumulated sums in registers, writes the bf16
-//            result into the tokens' slab rows and clears the accumulator. Without a shared
-//            expert combine_finalize_kernel does the last step.
+//            products; combine_finalize_kernel then writes every token's sum as bf16 into
+//            its slab row and clears the accumulator.
 #pragma once
 
 #include "ptx.cuh"
@@ -97,16 +91,8 @@ struct GemmParams {
   const int32_t* row_token;
   const float* row_w;
   float* acc;                 // [Tmax][H] fp32, zero between calls
-  // fused combine (layers with a shared expert): the shared expert's tiles finish each
-  // 128-token block x 256-column tile once its routed rows are in (see the epilogue)
-  int fuse_final;
-  const int32_t* tok_mt;      // [Tmax] (slab << 24) | row in slab
-  const int32_t* blk_need;    // [token blocks] target of each counter
-  int32_t* blk_cnt;           // [token blocks][n_tiles], zeroed by the routing
-  // split-K for launches whose tiles fill less than half of the grid: the K blocks of a
-  // tile are shared out among several CTAs. The down projection's partial sums go to the
-  // combine accumulators like any contribution (only without the fused combine); the gate
-  // / up projection's go to the fp32 workspace g_ws [g_rows][2I], and the CTA whose
+  // split-K for gate/up launches whose tiles fill less than half of the grid: the K blocks
+  // of a tile are shared out among several CTAs, whose partial sums go to the fp32 workspace g_ws [g_rows][2I], and the CTA whose
   // partial completes a tile's 32-row quadrant (g_cnt) finishes SwiGLU + requantisation
   // for those rows from it and clears it.
   int split_ok;
@@ -119,21 +105,16 @@ struct GemmParams {
 };
 
 constexpr int kMinSplitKb = 4;    // K blocks per split, at least
+constexpr int kMaxKb = AFD_MAX_QBLOCKS;   // K blocks of one projection (H/128, I/128)
 constexpr int kMaxSplits = 8;
 
 // 16-byte multiple: the combine staging that follows it is the source of bulk copies
-// Row scales of the A operand travel with the operands: for every K block the producer
-// bulk-copies the tile's 128 scales (from the 16-byte boundary at or below the tile's
-// first row: 132 floats) into a ring slot that the epilogue warps release after reading.
-constexpr int kScaleSlots = 8;                 // > stages + the MMA's lead over the epilogue
-constexpr int kScaleRowFloats = 132;
-constexpr uint32_t kScaleRowBytes = kScaleRowFloats * 4;
-static_assert(kScaleRowBytes % 16 == 0, "bulk copy size");
-
 struct alignas(16) GemmSmem {
-  float sring[kScaleSlots][kScaleRowFloats];   // first: 16-byte aligned rows
-  uint64_t sfull[kScaleSlots];
-  uint64_t sempty[kScaleSlots];
+  // weight-block scales of a tile: [slot][row][K block]; SWIGLU rows = gate, up block;
+  // COMBINE rows = the two 128-row halves of the 256 output columns
+  float wring[2][2][kMaxKb];
+  uint64_t wfull[2];
+  uint64_t wempty[2];
   uint64_t full[kMaxStages];
   uint64_t empty[kMaxStages];
   uint64_t tfull[2];
@@ -143,7 +124,6 @@ struct alignas(16) GemmSmem {
   int abort_flag;
   float amax[2][2][kTileM];
   int32_t mtile[AFD_MAX_GROUPS + 1];
-  int32_t pend[kEpiWarps][4];   // fused combine: {row0, rows, column tile} of a tile to count
 };
 static_assert(sizeof(GemmSmem) % 16 == 0, "staging after GemmSmem must stay 16-byte aligned");
 
@@ -233,34 +213,11 @@ __device__ __forceinline__ void split_swiglu_row(const GemmParams& p, int row, i
   p.sh_t[static_cast<size_t>(nt) * p.rpad + row] = sc;
 }
 
-// Fused combine: this thread's bulk reductions of a routed tile are performed; add its row
-// to the counter of (its token's 128-token block, the tile's column tile), with release
-// semantics, so that the shared tile that reads the block's sums sees them.
-// `pend` is the warp's {row0, rows, column tile} record in shared memory, cleared here.
-// The warp's rows are in token order, so they fall into one or a few token blocks: one
-// release-add per block, by the first lane of its run, after every lane has fenced its own
-// reductions (the warp barrier orders them before that add).
-__device__ __forceinline__ void combine_count(const GemmParams& p, int32_t* pend, int trow, int lane) {
-  const int row0 = pend[0], rows = pend[1], nt = pend[2];
-  bulk_wait_all();
-  fence_proxy_async_global();
-  __threadfence();
-  const int tb = trow < rows ? (p.row_token[row0 + trow] >> 7) : -1;
-  const unsigned same = __match_any_sync(0xffffffffu, tb);
-  __syncwarp();
-  if (tb >= 0 && lane == __ffs(same) - 1)
-    red_release_add(p.blk_cnt + static_cast<size_t>(tb) * p.n_tiles + nt, __popc(same));
-  __syncwarp();
-  if (lane == 0) pend[1] = 0;
-  __syncwarp();
-}
-
 template <int EPI>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ GemmParams p,
                         const __grid_constant__ CUtensorMap tm_a,
-                        const __grid_constant__ CUtensorMap tm_b,
-                        const __grid_constant__ YTable ytab) {
+                        const __grid_constant__ CUtensorMap tm_b) {
   constexpr int kStages = GemmCfg<EPI>::kStages;
 
   extern __shared__ uint8_t smem_raw[];
@@ -285,9 +242,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_init(&S.tempty[b], kEpiWarps);
     }
     for (int i = 0; i < 4; ++i) mbar_init(&S.pair[i], 64);
-    for (int i = 0; i < kScaleSlots; ++i) {
-      mbar_init(&S.sfull[i], 1);
-      mbar_init(&S.sempty[i], kEpiWarps);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&S.wfull[i], 2);
+      mbar_init(&S.wempty[i], kEpiWarps);
     }
     S.abort_flag = 0;
     fence_mbar_init();
@@ -302,11 +259,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = S.tmem_base;
   const int nkb = p.num_kb;
-  // split-K when the tiles fill less than half of the grid (small batches)
+  // split-K when the gate/up projection's tiles fill less than half of the grid (small
+  // batches; the down projection has H/256 column tiles per m-tile and is left whole)
   const int n_tiles0 = S.mtile[p.G] * p.n_tiles;
   int splits = 1;
-  if (p.split_ok && n_tiles0 > 0 && 2 * n_tiles0 <= static_cast<int>(gridDim.x) &&
-      (EPI == EPI_COMBINE || S.mtile[p.G] * kTileM <= p.g_rows))
+  if (EPI == EPI_SWIGLU && p.split_ok && n_tiles0 > 0 && 2 * n_tiles0 <= static_cast<int>(gridDim.x) &&
+      S.mtile[p.G] * kTileM <= p.g_rows)
     splits = max(1, min(min(static_cast<int>(gridDim.x) / n_tiles0, nkb / kMinSplitKb), kMaxSplits));
   const int total_units = n_tiles0 * splits;
 
@@ -349,15 +307,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             skipped = it;       // test hook: never fill this stage
             continue;
           }
-          // the A rows' scales of this K block into the next ring slot
-          const int ss = it % kScaleSlots;
-          if (!mbar_wait(&S.sempty[ss], ((it / kScaleSlots) & 1) ^ 1, abort_flag, p.status, p.wait_limit_ns)) {
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(&S.sfull[ss], kScaleRowBytes);
-          bulk_load(S.sring[ss], p.sa_t + static_cast<size_t>(kb) * p.rpad + (c.row0 & ~3), kScaleRowBytes,
-                    &S.sfull[ss]);
           uint8_t* a = sA + s * kABytes;
           uint8_t* b = sB + s * kBBytes;
           mbar_arrive_expect_tx(&S.full[s], kStageBytes);
@@ -367,15 +316,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
       }
       if (!ok) {
-        // wait (bounded) for copies that may still be landing on this CTA's barriers (a
-        // K block whose stage wait failed issued nothing; its scale copy may have landed)
+        // wait (bounded) for copies that may still be landing on this CTA's barriers
         for (int j = max(0, it - kStages); j < it; ++j) {
           if (j == skipped) continue;
           mbar_wait_drain(&S.full[j % kStages], (j / kStages) & 1, p.wait_limit_ns);
-        }
-        for (int j = max(0, it - kScaleSlots); j < it; ++j) {
-          if (j == skipped) continue;
-          mbar_wait_drain(&S.sfull[j % kScaleSlots], (j / kScaleSlots) & 1, p.wait_limit_ns);
         }
       }
     } else if (warp == 1 && lane == 0) {
@@ -414,6 +358,30 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int last = it - 1;
         mbar_wait_drain(&S.tfull[last & 1], (last >> 1) & 1, p.wait_limit_ns);
       }
+    } else if (warp == 2 || warp == 3) {
+      // ------------------------------------------------ weight-scale loader (64 threads)
+      // one tile ahead of the epilogue: the two weight-block scale rows of every tile this
+      // CTA runs, in the order it runs them
+      const int tl = threadIdx.x - 64;
+      int j = 0;
+      for (int u = blockIdx.x; u < total_units; u += gridDim.x, ++j) {
+        const int tile = u / splits;
+        const TileCoord c = decode_tile(tile, p.n_tiles, p.slice_first, S.mtile, p.G, p.group_off);
+        const int r0 = EPI == EPI_SWIGLU ? c.nt : 2 * c.nt;
+        const int r1 = EPI == EPI_SWIGLU ? p.I / 128 + c.nt : 2 * c.nt + 1;
+        const float* w0 = p.w_scale + (static_cast<size_t>(c.e) * p.ws_rows + r0) * nkb;
+        const float* w1 = p.w_scale + (static_cast<size_t>(c.e) * p.ws_rows + r1) * nkb;
+        const int slot = j & 1;
+        int got = 1;
+        if (lane == 0) got = mbar_wait(&S.wempty[slot], ((j >> 1) & 1) ^ 1, abort_flag, p.status, p.wait_limit_ns);
+        if (!__shfl_sync(0xffffffffu, got, 0)) break;
+        for (int i = tl; i < nkb; i += 64) {
+          S.wring[slot][0][i] = __ldg(w0 + i);
+          S.wring[slot][1][i] = __ldg(w1 + i);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.wfull[slot]);
+      }
     }
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kEpilogueRegs));
@@ -426,69 +394,46 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     int kbg = 0, titer = 0;
     bool ok = true;
     const uint64_t pol_acc = policy_evict_last();
-    // fused combine: the last routed tile whose rows are still to be counted (its row0,
-    // rows and column tile in S.pend[ew]; rows == 0: none)
-    int32_t* pend = S.pend[ew];
-    if (lane == 0) pend[1] = 0;
-    __syncwarp();
     for (int u = blockIdx.x; ok && u < total_units; u += gridDim.x, ++titer) {
       const int tile = u / splits, sp = u - tile * splits;
       const int kb0 = sp * nkb / splits, kb1 = (sp + 1) * nkb / splits;
       const TileCoord c = decode_tile(tile, p.n_tiles, p.slice_first, S.mtile, p.G, p.group_off);
       const int grow = c.row0 + trow;
       const bool valid = trow < c.rows;
-      const float* wsb = p.w_scale + static_cast<size_t>(c.e) * p.ws_rows * nkb;
-      int rs0, rs1, c0, c1;
+      int c0, c1;
       if (EPI == EPI_SWIGLU) {
-        rs0 = c.nt;
-        rs1 = p.I / 128 + c.nt;
         c0 = 64 * half;
         c1 = 128 + 64 * half;
       } else {
-        rs0 = rs1 = 2 * c.nt + half;
         c0 = 128 * half;
         c1 = 128 * half + 64;
       }
-      const float* ws0 = wsb + static_cast<size_t>(rs0) * nkb;
-      const float* ws1 = wsb + static_cast<size_t>(rs1) * nkb;
+      // this tile's weight-block scales, loaded by warps 2..3: SWIGLU gate row (s0) and up
+      // row (s1); COMBINE the row of this warp's 128 output columns (both)
+      const int wslot = titer & 1;
+      // every lane waits (acquire) before reading the slot the loader warps wrote
+      if (!__all_sync(0xffffffffu, mbar_wait(&S.wfull[wslot], (titer >> 1) & 1, abort_flag, p.status,
+                                            p.wait_limit_ns))) {
+        ok = false;
+        break;
+      }
+      const float* ws0 = S.wring[wslot][EPI == EPI_SWIGLU ? 0 : half];
+      const float* ws1 = S.wring[wslot][EPI == EPI_SWIGLU ? 1 : half];
       // acc[j] holds columns (2j, 2j+1) of this thread's 128: [0,32) from the first
       // 64-column group, [32,64) from the second
       float2 acc[64];
 #pragma unroll
       for (int i = 0; i < 64; ++i) acc[i] = make_float2(0.f, 0.f);
-      // weight-block scales of K block kb+2 are fetched while block kb is processed; the
-      // row scales come through the ring (this thread's is at its row's offset from the
-      // 16-byte boundary the producer copied from)
-      const int sofs = (c.row0 & 3) + trow;
-      float w0_n = __ldg(ws0 + kb0), w1_n = __ldg(ws1 + kb0);
-      float w0_n2 = 0.f, w1_n2 = 0.f;
-      if (kb0 + 1 < kb1) {
-        w0_n2 = __ldg(ws0 + kb0 + 1);
-        w1_n2 = __ldg(ws1 + kb0 + 1);
-      }
-      // the K block at which a pending count of the previous tile is taken
-      const int count_kb = kb0 + (kb1 - kb0 > 3 ? 3 : kb1 - kb0 - 1);
+      // the row scales of K block kb+2 are fetched while block kb is processed (their L2
+      // latency under the operand stream is longer than one K block)
+      const float* sap = p.sa_t + grow;
+      float sa_n = sap[static_cast<size_t>(kb0) * p.rpad];
+      float sa_n2 = kb0 + 1 < kb1 ? sap[static_cast<size_t>(kb0 + 1) * p.rpad] : 0.f;
       for (int kb = kb0; kb < kb1; ++kb, ++kbg) {
-        if (EPI == EPI_COMBINE && kb == count_kb && pend[1] > 0) {
-          // a few K blocks after they were issued the previous tile's reductions are done
-          combine_count(p, pend, trow, lane);
-        }
-        const int ss = kbg % kScaleSlots;
-        if (!mbar_wait(&S.sfull[ss], (kbg / kScaleSlots) & 1, abort_flag, p.status, p.wait_limit_ns)) {
-          ok = false;
-          break;
-        }
-        const float sa = S.sring[ss][sofs];
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&S.sempty[ss]);
-        const float s0 = sa * w0_n;
-        const float s1 = sa * w1_n;
-        w0_n = w0_n2;
-        w1_n = w1_n2;
-        if (kb + 2 < kb1) {
-          w0_n2 = __ldg(ws0 + kb + 2);
-          w1_n2 = __ldg(ws1 + kb + 2);
-        }
+        const float s0 = sa_n * ws0[kb];
+        const float s1 = sa_n * ws1[kb];
+        sa_n = sa_n2;
+        if (kb + 2 < kb1) sa_n2 = sap[static_cast<size_t>(kb + 2) * p.rpad];
         const int b = kbg & 1;
         const uint32_t tph = (kbg >> 1) & 1;
         int got = 1;
@@ -529,6 +474,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
       }
       if (!ok) break;
+      // the tile's weight scales are read: their slot may be refilled
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.wempty[wslot]);
 
       if (EPI == EPI_SWIGLU && splits > 1) {
         // this unit's partial sum into G; the warp whose partial completes the tile's
@@ -592,95 +540,38 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (half == 0) p.sh_t[static_cast<size_t>(c.nt) * p.rpad + grow] = sc;
         }
       } else {
+        // weighted combine: this warp's 32 rows x 128 columns, times each row's top-K
+        // weight, go to the token accumulators as bulk reductions (one 512-byte row
+        // segment each). Eight lanes at a time fill one of the warp's two staging buffers
+        // and issue their rows; before a buffer is refilled, the lanes that issued from it
+        // last wait until the bulk engine has read it.
         const int col0 = c.nt * kBN + half * 128;
-        if (pend[1] > 0) combine_count(p, pend, trow, lane);
-        if (!p.fuse_final || c.e != p.G - 1) {
-          // weighted combine: this warp's 32 rows x 128 columns, times each row's top-K
-          // weight, go to the token accumulators as bulk reductions (one 512-byte row
-          // segment each). Eight lanes at a time fill one of the warp's two staging buffers
-          // and issue their rows; before a buffer is refilled, the lanes that issued from
-          // it last wait until the bulk engine has read it.
-          int g = -1;
-          float wgt = 0.f;
-          if (valid) {
-            g = p.row_token[grow];
-            wgt = p.row_w[grow];
-          }
-          uint8_t* wst = stg + ew * kStgWarpBytes;
+        int g = -1;
+        float wgt = 0.f;
+        if (valid) {
+          g = p.row_token[grow];
+          wgt = p.row_w[grow];
+        }
+        uint8_t* wst = stg + ew * kStgWarpBytes;
 #pragma unroll
-          for (int r8 = 0; r8 < 4; ++r8) {
-            uint8_t* buf = wst + (r8 & 1) * kStgBufBytes;
-            if ((lane >> 3) == ((r8 + 2) & 3)) bulk_wait_read_all();
-            __syncwarp();
-            if ((lane >> 3) == r8) {
-              float* row = reinterpret_cast<float*>(buf + (lane & 7) * kStgRowBytes);
+        for (int r8 = 0; r8 < 4; ++r8) {
+          uint8_t* buf = wst + (r8 & 1) * kStgBufBytes;
+          if ((lane >> 3) == ((r8 + 2) & 3)) bulk_wait_read_all();
+          __syncwarp();
+          if ((lane >> 3) == r8) {
+            float* row = reinterpret_cast<float*>(buf + (lane & 7) * kStgRowBytes);
 #pragma unroll
-              for (int i = 0; i < 32; ++i) {
-                const float2 a = acc[2 * i], bb = acc[2 * i + 1];
-                *reinterpret_cast<float4*>(row + 4 * i) =
-                    make_float4(a.x * wgt, a.y * wgt, bb.x * wgt, bb.y * wgt);
-              }
-              fence_proxy_async_shared();
-              if (g >= 0)
-                bulk_reduce_add_f32(p.acc + static_cast<size_t>(g) * p.H + col0, row, 512, pol_acc);
-              bulk_commit();
+            for (int i = 0; i < 32; ++i) {
+              const float2 a = acc[2 * i], bb = acc[2 * i + 1];
+              *reinterpret_cast<float4*>(row + 4 * i) = make_float4(a.x * wgt, a.y * wgt, bb.x * wgt, bb.y * wgt);
             }
-          }
-          if (p.fuse_final) {
-            __syncwarp();
-            if (lane == 0) {
-              pend[0] = c.row0;
-              pend[1] = c.rows;
-              pend[2] = c.nt;
-            }
-            __syncwarp();
-          }
-        } else {
-          // the shared expert's tile of token block tb (its rows are the tokens 128 tb ..
-          // 128 tb + 127, weight 1): once the routed rows of the block are in, add this
-          // row to the accumulated sum, write bf16 into the token's slab row, clear the sum
-          const int tb = c.mt - S.mtile[p.G - 1];
-          const int* cnt = p.blk_cnt + static_cast<size_t>(tb) * p.n_tiles + c.nt;
-          const int target = p.blk_need[tb];
-          int got = 1;
-          if (lane == 0) got = wait_count(cnt, target, abort_flag, p.status, p.wait_limit_ns);
-          got = __shfl_sync(0xffffffffu, got, 0);
-          if (!got) {
-            ok = false;
-            break;
-          }
-          ld_acquire(cnt);
-          if (valid) {
-            const int g = 128 * tb + trow;
-            const int mt = p.tok_mt[g];
-            float* arow = p.acc + static_cast<size_t>(g) * p.H + col0;
-            uint4* yrow = reinterpret_cast<uint4*>(ytab.y[mt >> 24] + static_cast<size_t>(mt & 0xFFFFFF) * p.H + col0);
-#pragma unroll
-            for (int h4 = 0; h4 < 4; ++h4) {      // 32 columns at a time
-              float4 a[8];
-#pragma unroll
-              for (int i = 0; i < 8; ++i) a[i] = __ldcg(reinterpret_cast<const float4*>(arow + 32 * h4 + 4 * i));
-#pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                const float4 u = a[2 * i], v = a[2 * i + 1];
-                const float2 x0 = acc[16 * h4 + 4 * i], x1 = acc[16 * h4 + 4 * i + 1];
-                const float2 x2 = acc[16 * h4 + 4 * i + 2], x3 = acc[16 * h4 + 4 * i + 3];
-                uint4 o;
-                o.x = pack_bf16x2(u.x + x0.x, u.y + x0.y);
-                o.y = pack_bf16x2(u.z + x1.x, u.w + x1.y);
-                o.z = pack_bf16x2(v.x + x2.x, v.y + x2.y);
-                o.w = pack_bf16x2(v.z + x3.x, v.w + x3.y);
-                yrow[4 * h4 + i] = o;
-              }
-#pragma unroll
-              for (int i = 0; i < 8; ++i)
-                __stcg(reinterpret_cast<float4*>(arow + 32 * h4 + 4 * i), make_float4(0.f, 0.f, 0.f, 0.f));
-            }
+            fence_proxy_async_shared();
+            if (g >= 0) bulk_reduce_add_f32(p.acc + static_cast<size_t>(g) * p.H + col0, row, 512, pol_acc);
+            bulk_commit();
           }
         }
       }
     }
-    if (EPI == EPI_COMBINE && ok && pend[1] > 0) combine_count(p, pend, trow, lane);
     // every bulk reduction issued by this thread has been performed before the CTA exits
     if (EPI == EPI_COMBINE) bulk_wait_all();
   }

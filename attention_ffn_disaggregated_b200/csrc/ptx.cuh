@@ -307,41 +307,6 @@ __device__ __forceinline__ void fence_proxy_async_shared() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-// Cross-CTA counters (release / acquire at GPU scope).
-__device__ __forceinline__ void red_release_add(int* addr, int v) {
-  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(addr), "r"(v) : "memory");
-}
-__device__ __forceinline__ int ld_acquire(const int* addr) {
-  int v;
-  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(addr) : "memory");
-  return v;
-}
-// Bounded wait until *addr >= target; on expiry or a raised abort flag it behaves like
-// mbar_wait (flag and TIMEOUT status set, returns false).
-__device__ __forceinline__ bool wait_count(const int* addr, int target, volatile int* abort_flag,
-                                           int* status, uint64_t limit_ns) {
-  if (ld_acquire(addr) >= target) return true;
-  const uint64_t t0 = globaltimer_ns();
-  uint32_t n = 0;
-  while (true) {
-    __nanosleep(64);
-    if (ld_acquire(addr) >= target) return true;
-    if ((++n & 15u) == 0) {
-      if (*abort_flag) return false;
-      if (globaltimer_ns() - t0 > limit_ns) {
-        *abort_flag = 1;
-        atomicOr(status, AFD_STATUS_TIMEOUT);
-        return false;
-      }
-    }
-  }
-}
-// order this thread's completed bulk (async-proxy) global writes before its later
-// generic-proxy operations
-__device__ __forceinline__ void fence_proxy_async_global() {
-  asm volatile("fence.proxy.async.global;" ::: "memory");
-}
-
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);

@@ -43,12 +43,6 @@ struct RouteParams {
   int tiling;             // as set on the plan: 0 (default, = 1) .. 2; -1: routing only
   int32_t* tok_mt;        // [Tmax] (slab << 24) | row
   int32_t* tok_need;      // [Tmax] contributions this GPU adds to the token
-  // fused combine (layers with a shared expert; null otherwise): per 128-token block, the
-  // count the down projection's routed tiles reach (two per routed row: one per epilogue
-  // half), and the per (block, 256-column tile) counters they add to, zeroed here
-  int32_t* blk_need;      // [2 * num_chunks]
-  int32_t* blk_cnt;       // [2 * num_chunks][n_ctiles]
-  int n_ctiles;
   int32_t* pos;           // [Tmax*K]
   int32_t* row_token;     // [rpad]
   int32_t* row_k;         // [rpad]
@@ -201,7 +195,6 @@ __global__ void __launch_bounds__(kRouteThreads) route_count_kernel(
   for (int e = threadIdx.x; e < p.El; e += blockDim.x) s_hist[e] = 0;
   __syncthreads();
   const int g = blockIdx.x * kChunkTokens + threadIdx.x;
-  int routed = 0;
   if (g < T) {
     const int m = find_slab(s_base, p.M, g);
     const int t = g - s_base[m];
@@ -215,24 +208,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_count_kernel(
       if (mask >> k & 1u) atomicAdd(&s_hist[le[k]], 1);
     p.tok_mt[g] = (m << 24) | t;
     p.tok_need[g] = __popc(mask) + p.S;
-    routed = __popc(mask);
     if (bad) atomicOr(p.status, AFD_STATUS_BAD_ROUTING);
-  }
-  if (p.blk_need) {
-    // this CTA's two 128-token blocks: their targets and zeroed counters
-    static_assert(kChunkTokens == 256 && kRouteWarps == 8, "two 128-token blocks per routing CTA");
-    __shared__ int s_bn[kRouteWarps];
-    int v = routed;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    if ((threadIdx.x & 31) == 0) s_bn[threadIdx.x >> 5] = v;
-    const size_t tb0 = static_cast<size_t>(blockIdx.x) * 2;
-    for (int i = threadIdx.x; i < 2 * p.n_ctiles; i += blockDim.x) p.blk_cnt[tb0 * p.n_ctiles + i] = 0;
-    __syncthreads();
-    if (threadIdx.x < 2) {
-      const int* w = s_bn + 4 * threadIdx.x;
-      p.blk_need[tb0 + threadIdx.x] = 2 * (w[0] + w[1] + w[2] + w[3]);
-    }
   }
   __syncthreads();
   int32_t* out = p.chunk_hist + static_cast<size_t>(blockIdx.x) * max(p.El, 1);

@@ -79,12 +79,12 @@ typedef enum {
 #define AFD_MAX_TOP_K 32
 #define AFD_MAX_GROUPS 1024 /* num_local_experts + has_shared_expert */
 #define AFD_QBLOCK 128      /* quantisation block edge */
+#define AFD_MAX_QBLOCKS 128 /* hidden and intermediate are at most 128 blocks (16384) */
 
 /* Timed stages of one layer call, in launch order (for afd_ffn_get_kernel_times). One
  * kernel per stage, except that the routing scan runs in the last block of the route
  * count kernel (AFD_KERNEL_ROUTE_COUNT covers both and AFD_KERNEL_ROUTE_SCAN reads as
- * zero) and that with a shared expert the down projection writes the slab rows itself
- * (AFD_KERNEL_FINALIZE reads as zero). The gather stage copies the routed FP8 rows and their scales into expert order. */
+ * zero). The gather stage copies the routed FP8 rows and their scales into expert order. */
 #define AFD_KERNEL_ROUTE_COUNT 0
 #define AFD_KERNEL_ROUTE_SCAN 1
 #define AFD_KERNEL_ROUTE_SCATTER 2
@@ -101,8 +101,10 @@ typedef struct afd_ffn_plan_s* afd_ffn_plan_t; /* opaque; owned by the library *
 
 typedef struct {
   int32_t hidden;             /* H, multiple of 128; AFD_ERR_UNSUPPORTED unless a multiple
-                                 of 256 (the down projection writes 256-column tiles) */
-  int32_t intermediate;       /* I, multiple of 128 */
+                                 of 256 (the down projection writes 256-column tiles) and
+                                 at most 128 * AFD_MAX_QBLOCKS */
+  int32_t intermediate;       /* I, multiple of 128; AFD_ERR_UNSUPPORTED above
+                                 128 * AFD_MAX_QBLOCKS */
   int32_t num_experts_global; /* E_g >= 1: ids the router may emit are [0, E_g) */
   int32_t expert_begin;       /* e0 >= 0 */
   int32_t num_local_experts;  /* E_l >= 0, e0 + E_l <= E_g */
@@ -295,8 +297,7 @@ AFD_API afd_status_t afd_ffn_route_noalloc(const afd_ffn_config_t* cfg, const af
                                            afd_stream_t stream);
 
 /* Number of this library's kernel launches one afd_ffn_layer call of this plan makes with
- * its current tiling: 5 with a shared expert, 6 without (a separate finalisation writes the
- * slab rows), one more with tiling 2. -1 for NULL. */
+ * its current tiling: 6, one more with tiling 2. -1 for NULL. */
 AFD_API int32_t afd_ffn_kernels_per_layer(afd_ffn_plan_t plan);
 
 /* Human-readable name of a status code. */

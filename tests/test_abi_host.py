@@ -52,6 +52,7 @@ def _cfg(**kw):
     ({"num_slabs": 0}, 1), ({"num_slabs": 129}, 2), ({"slab_capacity": 0}, 1),
     ({"slab_capacity": 1 << 24}, 2),
     ({"num_experts_global": 2048, "num_local_experts": 1024, "has_shared_expert": 1}, 2),
+    ({"hidden": 16640}, 2), ({"intermediate": 16512}, 2),   # above 128 quantisation blocks
 ])
 def test_check_config_codes(kw, code):
     c = _cfg(**kw)

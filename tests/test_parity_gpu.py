@@ -55,10 +55,11 @@ def test_ragged_tiles_two_calls(seed, shape, counts, cap):
     assert res["status_rc"] == 0
 
 
-# Small batches: when a projection's tiles fill at most half of the GPU, each tile's K
-# blocks are shared out among CTAs (split-K). H = I = 1024 gives 8 K blocks per tile, so
-# both projections split in two; with a shared expert only W13 splits. Three calls check
-# that the split workspace and its counters are clear again after every call.
+# Small batches: when the gate/up projection's tiles fill at most half of the GPU, each
+# tile's K blocks are shared out among CTAs (split-K) and the CTA that completes a tile's
+# rows finishes SwiGLU + requantisation from the fp32 sums. H = 1024 or 2048 gives 8 or 16
+# K blocks per tile (two splits or more). Three calls check that the split workspace and
+# its counters are clear again after every call.
 @pytest.mark.parametrize("shape,counts,cap", [
     (W.LayerShape(1024, 1024, 8, 0, 8, 0, 2), [3], 3),
     (W.LayerShape(1024, 1024, 8, 0, 8, 0, 2), [1, 0, 16], 16),
