@@ -105,11 +105,12 @@ const char* afd_status_string(afd_status_t s) {
   return "unknown";
 }
 
-// route count (+ scan), scatter, gather, W13, W2, finalisation; the block-scale tiling
-// adds the activation factor images
+// route count (+ scan), scatter, gather, W13, W2, finalisation (a plan of at most
+// kSmallRouteChunks routing chunks runs the routing as one launch); the block-scale
+// tiling adds the activation factor images
 int32_t afd_ffn_kernels_per_layer(afd_ffn_plan_t P) {
   if (!P) return -1;
-  return 6 + (P->tiling == 2 ? 1 : 0);
+  return (P->num_chunks <= kSmallRouteChunks ? 5 : 6) + (P->tiling == 2 ? 1 : 0);
 }
 
 afd_status_t afd_ffn_check_config(const afd_ffn_config_t* c) {
@@ -308,6 +309,10 @@ afd_status_t afd_ffn_plan(const afd_ffn_config_t* cfg, const afd_ffn_weights_t* 
       cudaFuncSetAttribute(route_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(sizeof(int32_t) * (kRouteWarps * AFD_MAX_GROUPS +
                                                                kRouteWarps * 32 * AFD_MAX_TOP_K))) !=
+          cudaSuccess ||
+      cudaFuncSetAttribute(route_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(sizeof(int32_t) * (kRouteWarps * AFD_MAX_GROUPS +
+                                                               kRouteWarps * 32 * AFD_MAX_TOP_K))) !=
           cudaSuccess) {
     cudaGetLastError();
     cudaFree(P->ws);
@@ -457,11 +462,19 @@ afd_status_t afd_ffn_layer(afd_ffn_plan_t P, const afd_slab_t* slabs, const int3
 
   const bool tm = P->timing;
   if (tm) cudaEventRecord(P->ev[0], stream);
-  // the routing scan runs in route_count's last block (its stage time reads as zero)
-  route_count_kernel<<<P->num_chunks, kRouteThreads, 0, stream>>>(rp, tab);
-  if (tm) cudaEventRecord(P->ev[1], stream);
-  if (tm) cudaEventRecord(P->ev[2], stream);
-  route_scatter_kernel<<<P->num_chunks, kRouteThreads, P->scatter_smem, stream>>>(rp, tab);
+  if (P->num_chunks <= kSmallRouteChunks) {
+    // small plans: count, scan and scatter in one block (the scan and scatter stage times
+    // read as zero)
+    route_small_kernel<<<1, kRouteThreads, P->scatter_smem, stream>>>(rp, tab);
+    if (tm) cudaEventRecord(P->ev[1], stream);
+    if (tm) cudaEventRecord(P->ev[2], stream);
+  } else {
+    // the routing scan runs in route_count's last block (its stage time reads as zero)
+    route_count_kernel<<<P->num_chunks, kRouteThreads, 0, stream>>>(rp, tab);
+    if (tm) cudaEventRecord(P->ev[1], stream);
+    if (tm) cudaEventRecord(P->ev[2], stream);
+    route_scatter_kernel<<<P->num_chunks, kRouteThreads, P->scatter_smem, stream>>>(rp, tab);
+  }
   if (tm) cudaEventRecord(P->ev[3], stream);
   gather_rows_kernel<<<P->num_sms * 8, kRouteThreads, 0, stream>>>(rp, tab);
   if (tm) cudaEventRecord(P->ev[4], stream);

@@ -179,22 +179,15 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(const __grid_constant_
   route_scan_body(p, p.info[0], s_warp);
 }
 
-// 1. per-chunk histogram of local groups; token bookkeeping. With p.scan_ticket set, the
-// block that finishes last also runs step 2 (every block publishes its histogram, fences,
-// then takes a ticket; the counter is returned to zero for the next call).
-__global__ void __launch_bounds__(kRouteThreads) route_count_kernel(
-    const __grid_constant__ RouteParams p, const __grid_constant__ SlabTable slabs) {
-  __shared__ int32_t s_base[AFD_MAX_SLABS + 1];
-  __shared__ int32_t s_hist[AFD_MAX_GROUPS];
-  load_slab_base(p, s_base);
-  const int T = s_base[p.M];
-  if (blockIdx.x == 0) {
-    for (int m = threadIdx.x; m <= p.M; m += blockDim.x) p.slab_base[m] = s_base[m];
-    if (threadIdx.x == 0) p.info[0] = T;
-  }
+// 1 for one chunk of 256 tokens (thread = token): classification, histogram of the local
+// groups in shared memory, token bookkeeping; the histogram goes to chunk_hist[chunk].
+// Called by all threads of the block.
+__device__ __forceinline__ void route_count_chunk(const RouteParams& p, const SlabTable& slabs,
+                                                  const int32_t* s_base, int T, int chunk,
+                                                  int32_t* s_hist) {
   for (int e = threadIdx.x; e < p.El; e += blockDim.x) s_hist[e] = 0;
   __syncthreads();
-  const int g = blockIdx.x * kChunkTokens + threadIdx.x;
+  const int g = chunk * kChunkTokens + threadIdx.x;
   if (g < T) {
     const int m = find_slab(s_base, p.M, g);
     const int t = g - s_base[m];
@@ -211,8 +204,25 @@ __global__ void __launch_bounds__(kRouteThreads) route_count_kernel(
     if (bad) atomicOr(p.status, AFD_STATUS_BAD_ROUTING);
   }
   __syncthreads();
-  int32_t* out = p.chunk_hist + static_cast<size_t>(blockIdx.x) * max(p.El, 1);
+  int32_t* out = p.chunk_hist + static_cast<size_t>(chunk) * max(p.El, 1);
   for (int e = threadIdx.x; e < p.El; e += blockDim.x) out[e] = s_hist[e];
+  __syncthreads();   // s_hist is read above before a next chunk clears it
+}
+
+// 1. per-chunk histogram of local groups; token bookkeeping. With p.scan_ticket set, the
+// block that finishes last also runs step 2 (every block publishes its histogram, fences,
+// then takes a ticket; the counter is returned to zero for the next call).
+__global__ void __launch_bounds__(kRouteThreads) route_count_kernel(
+    const __grid_constant__ RouteParams p, const __grid_constant__ SlabTable slabs) {
+  __shared__ int32_t s_base[AFD_MAX_SLABS + 1];
+  __shared__ int32_t s_hist[AFD_MAX_GROUPS];
+  load_slab_base(p, s_base);
+  const int T = s_base[p.M];
+  if (blockIdx.x == 0) {
+    for (int m = threadIdx.x; m <= p.M; m += blockDim.x) p.slab_base[m] = s_base[m];
+    if (threadIdx.x == 0) p.info[0] = T;
+  }
+  route_count_chunk(p, slabs, s_base, T, blockIdx.x, s_hist);
   if (!p.scan_ticket) return;
   __shared__ int s_last;
   __shared__ int s_warp[32];
@@ -226,22 +236,18 @@ __global__ void __launch_bounds__(kRouteThreads) route_count_kernel(
   if (threadIdx.x == 0) *p.scan_ticket = 0;
 }
 
-// 3. stable placement of every local (token, slot) pair and of the shared rows.
-// Dynamic shared memory: s_run [warps][El] + s_key [warps][32*K] int32.
-__global__ void __launch_bounds__(kRouteThreads) route_scatter_kernel(
-    const __grid_constant__ RouteParams p, const __grid_constant__ SlabTable slabs) {
-  extern __shared__ int32_t s_dyn[];
-  __shared__ int32_t s_base[AFD_MAX_SLABS + 1];
+// 3 for one chunk: stable placement of its local (token, slot) pairs and of its tokens'
+// shared rows; zero output rows of its tokens that receive nothing. s_run [warps][El] and
+// s_key [warps][32*K] are shared memory. Called by all threads of the block.
+__device__ __forceinline__ void route_scatter_chunk(const RouteParams& p, const SlabTable& slabs,
+                                                    const int32_t* s_base, int T, int chunk,
+                                                    int32_t* s_run, int32_t* s_key) {
   const int El1 = max(p.El, 1);
-  int32_t* s_run = s_dyn;                                   // [warps][El1]
-  int32_t* s_key = s_dyn + kRouteWarps * El1;               // [warps][32*K]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int m = threadIdx.x; m <= p.M; m += blockDim.x) s_base[m] = p.slab_base[m];
   for (int i = threadIdx.x; i < kRouteWarps * El1; i += blockDim.x) s_run[i] = 0;
   __syncthreads();
-  const int T = s_base[p.M];
   const int K = p.K;
-  const int g = blockIdx.x * kChunkTokens + warp * kTokensPerWarp + lane;
+  const int g = chunk * kChunkTokens + warp * kTokensPerWarp + lane;
   int m = 0, t = 0;
   int32_t* mykeys = s_key + warp * 32 * K;
   if (g < T) {
@@ -262,7 +268,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_scatter_kernel(
   }
   __syncthreads();
   // per-warp starting row of every group: group base + chunk base + earlier warps
-  const int32_t* coff = p.chunk_off + static_cast<size_t>(blockIdx.x) * El1;
+  const int32_t* coff = p.chunk_off + static_cast<size_t>(chunk) * El1;
   for (int e = threadIdx.x; e < p.El; e += blockDim.x) {
     int run = p.group_off[e] + coff[e];
     for (int w = 0; w < kRouteWarps; ++w) {
@@ -273,7 +279,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_scatter_kernel(
   }
   __syncthreads();
   // walk this warp's pairs in (token, slot) order, 32 at a time
-  const int gw0 = blockIdx.x * kChunkTokens + warp * kTokensPerWarp;
+  const int gw0 = chunk * kChunkTokens + warp * kTokensPerWarp;
   for (int r = 0; r < K; ++r) {
     const int pidx = r * 32 + lane;             // pair index inside the warp
     const int tl = pidx / K, k = pidx - tl * K;
@@ -317,6 +323,43 @@ __global__ void __launch_bounds__(kRouteThreads) route_scatter_kernel(
       for (int i = lane; i < p.H / 8; i += 32) dst[i] = make_uint4(0, 0, 0, 0);
     }
   }
+  __syncthreads();
+}
+
+// 3. stable placement of every local (token, slot) pair and of the shared rows, one
+// chunk per block. Dynamic shared memory: s_run [warps][El] + s_key [warps][32*K] int32.
+__global__ void __launch_bounds__(kRouteThreads) route_scatter_kernel(
+    const __grid_constant__ RouteParams p, const __grid_constant__ SlabTable slabs) {
+  extern __shared__ int32_t s_dyn[];
+  __shared__ int32_t s_base[AFD_MAX_SLABS + 1];
+  for (int m = threadIdx.x; m <= p.M; m += blockDim.x) s_base[m] = p.slab_base[m];
+  __syncthreads();
+  route_scatter_chunk(p, slabs, s_base, s_base[p.M], blockIdx.x, s_dyn,
+                      s_dyn + kRouteWarps * max(p.El, 1));
+}
+
+// 1-3 in one block for small plans (one chunk, at most 256 tokens): the chunk's counts,
+// the scan and the chunk's placement in sequence, without the launches and the global
+// round trips between them. The same per-chunk code, so the same routing bit for bit.
+// (With two chunks or more the chunks' work in one block outweighs the saved launch.)
+constexpr int kSmallRouteChunks = 1;
+__global__ void __launch_bounds__(kRouteThreads) route_small_kernel(
+    const __grid_constant__ RouteParams p, const __grid_constant__ SlabTable slabs) {
+  extern __shared__ int32_t s_dyn[];
+  __shared__ int32_t s_base[AFD_MAX_SLABS + 1];
+  __shared__ int32_t s_hist[AFD_MAX_GROUPS];
+  __shared__ int s_warp[32];
+  load_slab_base(p, s_base);
+  const int T = s_base[p.M];
+  for (int m = threadIdx.x; m <= p.M; m += blockDim.x) p.slab_base[m] = s_base[m];
+  if (threadIdx.x == 0) p.info[0] = T;
+  const int chunks = (T + kChunkTokens - 1) / kChunkTokens;
+  for (int c = 0; c < chunks; ++c) route_count_chunk(p, slabs, s_base, T, c, s_hist);
+  __syncthreads();
+  route_scan_body(p, T, s_warp);
+  __syncthreads();
+  for (int c = 0; c < chunks; ++c)
+    route_scatter_chunk(p, slabs, s_base, T, c, s_dyn, s_dyn + kRouteWarps * max(p.El, 1));
 }
 
 // 4. copy routed rows (FP8 codes and their per-128 scales) into expert order.

@@ -99,6 +99,7 @@ KERNEL_SOURCES = {
     "gather_rows": _ROUTE_SRC,
     "route_count": _ROUTE_SRC,
     "route_scatter": _ROUTE_SRC,
+    "route_small": _ROUTE_SRC,
 }
 
 

@@ -84,7 +84,8 @@ typedef enum {
 /* Timed stages of one layer call, in launch order (for afd_ffn_get_kernel_times). One
  * kernel per stage, except that the routing scan runs in the last block of the route
  * count kernel (AFD_KERNEL_ROUTE_COUNT covers both and AFD_KERNEL_ROUTE_SCAN reads as
- * zero). The gather stage copies the routed FP8 rows and their scales into expert order. */
+ * zero), and that a plan of at most 256 tokens (num_slabs * slab_capacity) routes in one
+ * block (AFD_KERNEL_ROUTE_COUNT covers count, scan and scatter). The gather stage copies the routed FP8 rows and their scales into expert order. */
 #define AFD_KERNEL_ROUTE_COUNT 0
 #define AFD_KERNEL_ROUTE_SCAN 1
 #define AFD_KERNEL_ROUTE_SCATTER 2
@@ -297,7 +298,8 @@ AFD_API afd_status_t afd_ffn_route_noalloc(const afd_ffn_config_t* cfg, const af
                                            afd_stream_t stream);
 
 /* Number of this library's kernel launches one afd_ffn_layer call of this plan makes with
- * its current tiling: 6, one more with tiling 2. -1 for NULL. */
+ * its current tiling: 6, or 5 when num_slabs * slab_capacity <= 256 (the routing runs in
+ * one block), one more with tiling 2. -1 for NULL. */
 AFD_API int32_t afd_ffn_kernels_per_layer(afd_ffn_plan_t plan);
 
 /* Human-readable name of a status code. */
