@@ -297,7 +297,7 @@ afd_status_t afd_ffn_plan(const afd_ffn_config_t* cfg, const afd_ffn_weights_t* 
     delete P;
     return st;
   }
-  P->scatter_smem = sizeof(int32_t) * (static_cast<size_t>(kRouteWarps) * El1 + kRouteWarps * 32 * K);
+  P->scatter_smem = scatter_smem_bytes(El1, K);
   if (cudaFuncSetAttribute(w13_mx_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(mx_smem_bytes())) != cudaSuccess ||
       cudaFuncSetAttribute(grouped_gemm_kernel<EPI_SWIGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -307,12 +307,10 @@ afd_status_t afd_ffn_plan(const afd_ffn_config_t* cfg, const afd_ffn_weights_t* 
       // the limit is a per-function setting shared by every plan: set the largest any
       // configuration can need, so that a later plan never lowers an earlier plan's limit
       cudaFuncSetAttribute(route_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(sizeof(int32_t) * (kRouteWarps * AFD_MAX_GROUPS +
-                                                               kRouteWarps * 32 * AFD_MAX_TOP_K))) !=
+                           static_cast<int>(scatter_smem_bytes(AFD_MAX_GROUPS, AFD_MAX_TOP_K))) !=
           cudaSuccess ||
       cudaFuncSetAttribute(route_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(sizeof(int32_t) * (kRouteWarps * AFD_MAX_GROUPS +
-                                                               kRouteWarps * 32 * AFD_MAX_TOP_K))) !=
+                           static_cast<int>(scatter_smem_bytes(AFD_MAX_GROUPS, AFD_MAX_TOP_K))) !=
           cudaSuccess) {
     cudaGetLastError();
     cudaFree(P->ws);
@@ -421,7 +419,7 @@ static void fill_gemm_params(afd_ffn_plan_t P, int epi, GemmParams& gp) {
     gp.row_w = P->row_w;
     gp.acc = P->acc;
     gp.slice_first = P->w2_slice_first;
-    gp.split_ok = 0;
+    gp.split_ok = 1;
   }
 }
 
@@ -666,8 +664,7 @@ afd_status_t noalloc_setup(int dev, uint8_t** out) {
       return AFD_ERR_CUDA;
     }
     if (cudaFuncSetAttribute(route_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(sizeof(int32_t) * (kRouteWarps * AFD_MAX_GROUPS +
-                                                                 kRouteWarps * 32 * AFD_MAX_TOP_K))) !=
+                             static_cast<int>(scatter_smem_bytes(AFD_MAX_GROUPS, AFD_MAX_TOP_K))) !=
         cudaSuccess) {
       cudaGetLastError();
       return AFD_ERR_CUDA;
@@ -759,8 +756,7 @@ extern "C" afd_status_t afd_ffn_route_noalloc(const afd_ffn_config_t* cfg, const
   rp.tiling = -1;           // routing only: d_sizes[3] = 0
   // every scratch region is fully written before it is read; only the status starts at 0
   if (cudaMemsetAsync(d_status, 0, sizeof(int32_t), stream) != cudaSuccess) return AFD_ERR_CUDA;
-  const size_t scatter_smem = sizeof(int32_t) * (static_cast<size_t>(kRouteWarps) * El1 +
-                                                 kRouteWarps * 32 * c.top_k);
+  const size_t scatter_smem = scatter_smem_bytes(El1, c.top_k);
   route_count_kernel<<<static_cast<int>(chunks), kRouteThreads, 0, stream>>>(rp, tab);
   route_scan_kernel<<<1, 1024, 0, stream>>>(rp);
   route_scatter_kernel<<<static_cast<int>(chunks), kRouteThreads, scatter_smem, stream>>>(rp, tab);

@@ -184,33 +184,46 @@ __device__ __forceinline__ float silu_mul(float g, float u) {
   return __fdividef(gx, 1.0f + __expf(-gx)) * u;
 }
 
-// Split-K W13: one row's SwiGLU + requantisation for intermediate block nt from the fp32
-// sums in G (gate at columns nt*128.., up at I + nt*128..), which are then cleared. The same
-// arithmetic as the one-CTA epilogue, with the row's 128 channels in one thread.
-__device__ __forceinline__ void split_swiglu_row(const GemmParams& p, int row, int nt) {
-  float* gr = p.g_ws + static_cast<size_t>(row) * (2 * p.I) + nt * 128;
-  // two passes over the row's sums in L2: the block amax, then the codes
-  float amax = 0.f;
-#pragma unroll 4
-  for (int i = 0; i < 32; ++i) {
-    const float4 g = __ldcg(reinterpret_cast<const float4*>(gr + 4 * i));
-    const float4 u = __ldcg(reinterpret_cast<const float4*>(gr + p.I + 4 * i));
-    amax = fmaxf(amax, fmaxf(fmaxf(fabsf(silu_mul(g.x, u.x)), fabsf(silu_mul(g.y, u.y))),
-                             fmaxf(fabsf(silu_mul(g.z, u.z)), fabsf(silu_mul(g.w, u.w)))));
+// Split-K W13: SwiGLU + requantisation of intermediate block nt for `nrows` consecutive
+// rows from `row0`, from the fp32 sums in G (gate at columns nt*128.., up at I + nt*128..),
+// which are then cleared. The whole warp works on four rows at a time (lane = 4 channels
+// of each), so a few rows cost one round trip to L2 rather than one per 4 channels. The
+// same arithmetic as the one-CTA epilogue; the block amax is a warp max.
+__device__ __forceinline__ void split_swiglu_rows(const GemmParams& p, int row0, int nrows, int nt,
+                                                  int lane) {
+  for (int r0 = 0; r0 < nrows; r0 += 4) {
+    float4 gv[4], uv[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if (r0 + j < nrows) {
+        const float* gr = p.g_ws + static_cast<size_t>(row0 + r0 + j) * (2 * p.I) + nt * 128 + 4 * lane;
+        gv[j] = __ldcg(reinterpret_cast<const float4*>(gr));
+        uv[j] = __ldcg(reinterpret_cast<const float4*>(gr + p.I));
+      } else {
+        gv[j] = uv[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float h0 = silu_mul(gv[j].x, uv[j].x), h1 = silu_mul(gv[j].y, uv[j].y);
+      const float h2 = silu_mul(gv[j].z, uv[j].z), h3 = silu_mul(gv[j].w, uv[j].w);
+      float amax = fmaxf(fmaxf(fabsf(h0), fabsf(h1)), fmaxf(fabsf(h2), fabsf(h3)));
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+      if (r0 + j < nrows) {
+        const int row = row0 + r0 + j;
+        const float sc = amax > 0.f ? amax / 448.0f : 1.0f;
+        const float rsc = __frcp_rn(sc);
+        uint32_t* dst = reinterpret_cast<uint32_t*>(p.hq + static_cast<size_t>(row) * p.I + nt * 128);
+        dst[lane] = static_cast<uint32_t>(pack_e4m3x2(h0 * rsc, h1 * rsc)) |
+                    (static_cast<uint32_t>(pack_e4m3x2(h2 * rsc, h3 * rsc)) << 16);
+        float* gr = p.g_ws + static_cast<size_t>(row) * (2 * p.I) + nt * 128 + 4 * lane;
+        __stcg(reinterpret_cast<float4*>(gr), make_float4(0.f, 0.f, 0.f, 0.f));
+        __stcg(reinterpret_cast<float4*>(gr + p.I), make_float4(0.f, 0.f, 0.f, 0.f));
+        if (lane == 0) p.sh_t[static_cast<size_t>(nt) * p.rpad + row] = sc;
+      }
+    }
   }
-  const float sc = amax > 0.f ? amax / 448.0f : 1.0f;
-  const float rsc = __frcp_rn(sc);
-  uint32_t* dst = reinterpret_cast<uint32_t*>(p.hq + static_cast<size_t>(row) * p.I + nt * 128);
-#pragma unroll 4
-  for (int i = 0; i < 32; ++i) {
-    const float4 g = __ldcg(reinterpret_cast<const float4*>(gr + 4 * i));
-    const float4 u = __ldcg(reinterpret_cast<const float4*>(gr + p.I + 4 * i));
-    dst[i] = static_cast<uint32_t>(pack_e4m3x2(silu_mul(g.x, u.x) * rsc, silu_mul(g.y, u.y) * rsc)) |
-             (static_cast<uint32_t>(pack_e4m3x2(silu_mul(g.z, u.z) * rsc, silu_mul(g.w, u.w) * rsc)) << 16);
-    __stcg(reinterpret_cast<float4*>(gr + 4 * i), make_float4(0.f, 0.f, 0.f, 0.f));
-    __stcg(reinterpret_cast<float4*>(gr + p.I + 4 * i), make_float4(0.f, 0.f, 0.f, 0.f));
-  }
-  p.sh_t[static_cast<size_t>(nt) * p.rpad + row] = sc;
 }
 
 template <int EPI>
@@ -259,12 +272,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = S.tmem_base;
   const int nkb = p.num_kb;
-  // split-K when the gate/up projection's tiles fill less than half of the grid (small
-  // batches; the down projection has H/256 column tiles per m-tile and is left whole)
+  // split-K when the tiles fill at most half of the grid (small batches). W13's splits
+  // meet in the fp32 workspace G and the last one finishes the tile; W2's partial sums
+  // are reduced into the token accumulators like whole tiles, so they need nothing more.
   const int n_tiles0 = S.mtile[p.G] * p.n_tiles;
   int splits = 1;
-  if (EPI == EPI_SWIGLU && p.split_ok && n_tiles0 > 0 && 2 * n_tiles0 <= static_cast<int>(gridDim.x) &&
-      S.mtile[p.G] * kTileM <= p.g_rows)
+  if (p.split_ok && n_tiles0 > 0 && 2 * n_tiles0 <= static_cast<int>(gridDim.x) &&
+      (EPI == EPI_COMBINE || S.mtile[p.G] * kTileM <= p.g_rows))
     splits = max(1, min(min(static_cast<int>(gridDim.x) / n_tiles0, nkb / kMinSplitKb), kMaxSplits));
   const int total_units = n_tiles0 * splits;
 
@@ -502,7 +516,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         old = __shfl_sync(0xffffffffu, old, 0);
         if (old == 2 * splits - 1) {
           __threadfence();
-          if (valid) split_swiglu_row(p, grow, c.nt);
+          split_swiglu_rows(p, c.row0 + 32 * q, min(32, max(0, c.rows - 32 * q)), c.nt, lane);
           __syncwarp();
           if (lane == 0) *cnt = 0;          // zero again for the next call
         }
@@ -590,31 +604,35 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 }
 
 // Combine, last step: every token's fp32 sum -> bf16 into its slab row; the accumulator
-// is cleared for the next call. One warp per token row, 16-byte stores.
+// is cleared for the next call. One warp per (token row, 256-column segment), 16-byte
+// stores, so that a few tokens still spread over many warps (the row's segments are
+// independent requests, not a chain of them).
 __global__ void __launch_bounds__(256) combine_finalize_kernel(const int32_t* __restrict__ info,
                                                                const int32_t* __restrict__ tok_mt,
                                                                float* __restrict__ acc, int H,
                                                                const __grid_constant__ YTable ytab) {
   const int T = info[0];
   const int lane = threadIdx.x & 31;
+  const int nseg = H / 256;                 // H is a multiple of 256
+  const int items = T * nseg;
   const int nwarps = (gridDim.x * blockDim.x) >> 5;
-  for (int g = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; g < T; g += nwarps) {
+  for (int it = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; it < items; it += nwarps) {
+    const int g = it / nseg;
+    const int c = (it - g * nseg) * 256 + lane * 8;
     const int mt = tok_mt[g];
     const int m = mt >> 24, t = mt & 0xFFFFFF;
     float* row = acc + static_cast<size_t>(g) * H;
     __nv_bfloat16* y = ytab.y[m] + static_cast<size_t>(t) * H;
-    for (int c = lane * 8; c < H; c += 256) {
-      const float4 a = __ldcg(reinterpret_cast<const float4*>(row + c));
-      const float4 b = __ldcg(reinterpret_cast<const float4*>(row + c + 4));
-      uint4 o;
-      o.x = pack_bf16x2(a.x, a.y);
-      o.y = pack_bf16x2(a.z, a.w);
-      o.z = pack_bf16x2(b.x, b.y);
-      o.w = pack_bf16x2(b.z, b.w);
-      *reinterpret_cast<uint4*>(y + c) = o;
-      __stcg(reinterpret_cast<float4*>(row + c), make_float4(0.f, 0.f, 0.f, 0.f));
-      __stcg(reinterpret_cast<float4*>(row + c + 4), make_float4(0.f, 0.f, 0.f, 0.f));
-    }
+    const float4 a = __ldcg(reinterpret_cast<const float4*>(row + c));
+    const float4 b = __ldcg(reinterpret_cast<const float4*>(row + c + 4));
+    uint4 o;
+    o.x = pack_bf16x2(a.x, a.y);
+    o.y = pack_bf16x2(a.z, a.w);
+    o.z = pack_bf16x2(b.x, b.y);
+    o.w = pack_bf16x2(b.z, b.w);
+    *reinterpret_cast<uint4*>(y + c) = o;
+    __stcg(reinterpret_cast<float4*>(row + c), make_float4(0.f, 0.f, 0.f, 0.f));
+    __stcg(reinterpret_cast<float4*>(row + c + 4), make_float4(0.f, 0.f, 0.f, 0.f));
   }
 }
 

@@ -237,11 +237,12 @@ __global__ void __launch_bounds__(kRouteThreads) route_count_kernel(
 }
 
 // 3 for one chunk: stable placement of its local (token, slot) pairs and of its tokens'
-// shared rows; zero output rows of its tokens that receive nothing. s_run [warps][El] and
-// s_key [warps][32*K] are shared memory. Called by all threads of the block.
+// shared rows; zero output rows of its tokens that receive nothing. s_run [warps][El],
+// s_key [warps][32*K] and s_wt [warps][32*K] are shared memory (the pairs' groups and
+// top-K weights, read once per token with its ids). Called by all threads of the block.
 __device__ __forceinline__ void route_scatter_chunk(const RouteParams& p, const SlabTable& slabs,
                                                     const int32_t* s_base, int T, int chunk,
-                                                    int32_t* s_run, int32_t* s_key) {
+                                                    int32_t* s_run, int32_t* s_key, float* s_wt) {
   const int El1 = max(p.El, 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int i = threadIdx.x; i < kRouteWarps * El1; i += blockDim.x) s_run[i] = 0;
@@ -250,13 +251,18 @@ __device__ __forceinline__ void route_scatter_chunk(const RouteParams& p, const 
   const int g = chunk * kChunkTokens + warp * kTokensPerWarp + lane;
   int m = 0, t = 0;
   int32_t* mykeys = s_key + warp * 32 * K;
+  float* mywt = s_wt + warp * 32 * K;
   if (g < T) {
     m = find_slab(s_base, p.M, g);
     t = g - s_base[m];
     int32_t ids[AFD_MAX_TOP_K];
     int le[AFD_MAX_TOP_K];
     const int32_t* src = slabs.ids[m] + static_cast<size_t>(t) * K;
-    for (int k = 0; k < K; ++k) ids[k] = src[k];
+    const float* wsrc = slabs.w[m] + static_cast<size_t>(t) * K;
+    for (int k = 0; k < K; ++k) {
+      ids[k] = src[k];
+      mywt[lane * K + k] = wsrc[k];
+    }
     bool bad = false;
     classify_token(ids, K, p.e0, p.El, p.Eg, le, &bad);
     for (int k = 0; k < K; ++k) {
@@ -289,12 +295,10 @@ __device__ __forceinline__ void route_scatter_chunk(const RouteParams& p, const 
       const int rank = __popc(peers & lanemask_lt());
       const int row = s_run[warp * El1 + key] + rank;
       const int gg = gw0 + tl;
-      const int mm = find_slab(s_base, p.M, gg);
-      const int tt = gg - s_base[mm];
       p.pos[static_cast<size_t>(gg) * K + k] = row;
       p.row_token[row] = gg;
       p.row_k[row] = k;
-      p.row_w[row] = slabs.w[mm][static_cast<size_t>(tt) * K + k];
+      p.row_w[row] = mywt[pidx];
     } else {
       const int gg = gw0 + tl;
       if (gg < T) p.pos[static_cast<size_t>(gg) * K + k] = -1;
@@ -326,40 +330,182 @@ __device__ __forceinline__ void route_scatter_chunk(const RouteParams& p, const 
   __syncthreads();
 }
 
+// Dynamic shared memory of the placement: s_run [warps][El] int32, s_key [warps][32*K]
+// int32, s_wt [warps][32*K] float.
+__host__ __device__ constexpr size_t scatter_smem_bytes(int El, int K) {
+  return sizeof(int32_t) * (static_cast<size_t>(kRouteWarps) * (El > 1 ? El : 1) +
+                            2 * static_cast<size_t>(kRouteWarps) * 32 * K);
+}
+
 // 3. stable placement of every local (token, slot) pair and of the shared rows, one
-// chunk per block. Dynamic shared memory: s_run [warps][El] + s_key [warps][32*K] int32.
+// chunk per block.
 __global__ void __launch_bounds__(kRouteThreads) route_scatter_kernel(
     const __grid_constant__ RouteParams p, const __grid_constant__ SlabTable slabs) {
   extern __shared__ int32_t s_dyn[];
   __shared__ int32_t s_base[AFD_MAX_SLABS + 1];
   for (int m = threadIdx.x; m <= p.M; m += blockDim.x) s_base[m] = p.slab_base[m];
   __syncthreads();
-  route_scatter_chunk(p, slabs, s_base, s_base[p.M], blockIdx.x, s_dyn,
-                      s_dyn + kRouteWarps * max(p.El, 1));
+  int32_t* s_key = s_dyn + kRouteWarps * max(p.El, 1);
+  route_scatter_chunk(p, slabs, s_base, s_base[p.M], blockIdx.x, s_dyn, s_key,
+                      reinterpret_cast<float*>(s_key + kRouteWarps * 32 * p.K));
 }
 
-// 1-3 in one block for small plans (one chunk, at most 256 tokens): the chunk's counts,
-// the scan and the chunk's placement in sequence, without the launches and the global
-// round trips between them. The same per-chunk code, so the same routing bit for bit.
-// (With two chunks or more the chunks' work in one block outweighs the saved launch.)
+// 1-3 in one block for one-chunk plans (at most 256 tokens, thread = token). The slab
+// counts are loaded in parallel and scanned; every token's ids and weights are read once;
+// the histogram, the group scan and the running rows stay in shared memory, so the block
+// waits on two global round trips (counts, then ids and weights) instead of one per step.
+// The placement is route_scatter_chunk's (per-warp counts, then ranks inside the warp in
+// (token, slot) order), so the routing is the same bit for bit.
 constexpr int kSmallRouteChunks = 1;
 __global__ void __launch_bounds__(kRouteThreads) route_small_kernel(
     const __grid_constant__ RouteParams p, const __grid_constant__ SlabTable slabs) {
   extern __shared__ int32_t s_dyn[];
   __shared__ int32_t s_base[AFD_MAX_SLABS + 1];
-  __shared__ int32_t s_hist[AFD_MAX_GROUPS];
+  __shared__ int32_t s_goff[AFD_MAX_GROUPS + 1];
   __shared__ int s_warp[32];
-  load_slab_base(p, s_base);
-  const int T = s_base[p.M];
-  for (int m = threadIdx.x; m <= p.M; m += blockDim.x) p.slab_base[m] = s_base[m];
-  if (threadIdx.x == 0) p.info[0] = T;
-  const int chunks = (T + kChunkTokens - 1) / kChunkTokens;
-  for (int c = 0; c < chunks; ++c) route_count_chunk(p, slabs, s_base, T, c, s_hist);
+  const int El1 = max(p.El, 1);
+  const int K = p.K;
+  int32_t* s_run = s_dyn;                         // [warps][El]
+  int32_t* s_key = s_dyn + kRouteWarps * El1;     // [warps][32*K]
+  float* s_wt = reinterpret_cast<float*>(s_key + kRouteWarps * 32 * K);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  // slab bases: one count per thread (M <= 128), clamped, block scan
+  int n = 0;
+  if (tid < p.M) {
+    n = p.counts[tid];
+    if (n < 0 || n > p.cap) {
+      atomicOr(p.status, AFD_STATUS_BAD_COUNT);
+      n = n < 0 ? 0 : p.cap;
+    }
+  }
+  for (int i = tid; i < kRouteWarps * El1; i += blockDim.x) s_run[i] = 0;
+  int T;
+  const int ex = block_exclusive_scan(n, s_warp, &T);
+  if (tid < p.M) {
+    s_base[tid] = ex;
+    p.slab_base[tid] = ex;
+  }
+  if (tid == 0) {
+    s_base[p.M] = T;
+    p.slab_base[p.M] = T;
+    p.info[0] = T;
+  }
   __syncthreads();
-  route_scan_body(p, T, s_warp);
+
+  // tokens: ids and weights, classification, per-warp group counts, token bookkeeping
+  const int g = tid;
+  int m = 0, t = 0, need = 0;
+  int32_t* mykeys = s_key + warp * 32 * K;
+  float* mywt = s_wt + warp * 32 * K;
+  if (g < T) {
+    m = find_slab(s_base, p.M, g);
+    t = g - s_base[m];
+    int32_t ids[AFD_MAX_TOP_K];
+    int le[AFD_MAX_TOP_K];
+    const int32_t* src = slabs.ids[m] + static_cast<size_t>(t) * K;
+    const float* wsrc = slabs.w[m] + static_cast<size_t>(t) * K;
+    for (int k = 0; k < K; ++k) {
+      ids[k] = src[k];
+      mywt[lane * K + k] = wsrc[k];
+    }
+    bool bad = false;
+    const uint32_t mask = classify_token(ids, K, p.e0, p.El, p.Eg, le, &bad);
+    for (int k = 0; k < K; ++k) {
+      mykeys[lane * K + k] = le[k];
+      if (le[k] >= 0) atomicAdd(&s_run[warp * El1 + le[k]], 1);
+    }
+    need = __popc(mask) + p.S;
+    p.tok_mt[g] = (m << 24) | t;
+    p.tok_need[g] = need;
+    if (bad) atomicOr(p.status, AFD_STATUS_BAD_ROUTING);
+  } else {
+    for (int k = 0; k < K; ++k) mykeys[lane * K + k] = -1;
+  }
   __syncthreads();
-  for (int c = 0; c < chunks; ++c)
-    route_scatter_chunk(p, slabs, s_base, T, c, s_dyn, s_dyn + kRouteWarps * max(p.El, 1));
+
+  // group counts, offsets and the m-tile schedule (exclusive scans over the groups)
+  int base_rows = 0, base_tiles = 0;
+  for (int g0 = 0; g0 < p.G; g0 += blockDim.x) {
+    const int e = g0 + tid;
+    int cnt = 0;
+    if (e < p.El) {
+      for (int w = 0; w < kRouteWarps; ++w) cnt += s_run[w * El1 + e];
+    } else if (e < p.G) {
+      cnt = T;                                    // the shared expert: every token
+    }
+    if (e < p.G) p.group_count[e] = cnt;
+    int tot_rows, tot_tiles;
+    const int ex_rows = block_exclusive_scan(cnt, s_warp, &tot_rows);
+    const int ex_tiles = block_exclusive_scan((cnt + kTileM - 1) / kTileM, s_warp, &tot_tiles);
+    if (e < p.G) {
+      s_goff[e] = base_rows + ex_rows;
+      p.group_off[e] = base_rows + ex_rows;
+      p.mtile_off[e] = base_tiles + ex_tiles;
+    }
+    base_rows += tot_rows;
+    base_tiles += tot_tiles;
+  }
+  if (tid == 0) {
+    s_goff[p.G] = base_rows;
+    p.group_off[p.G] = base_rows;
+    p.mtile_off[p.G] = base_tiles;
+    p.info[1] = base_rows;
+    p.info[2] = base_tiles;
+    p.info[3] = p.tiling < 0 ? 0 : (p.tiling == 0 ? 1 : p.tiling);
+  }
+  __syncthreads();
+  // per-warp starting row of every group
+  for (int e = tid; e < p.El; e += blockDim.x) {
+    int run = s_goff[e];
+    for (int w = 0; w < kRouteWarps; ++w) {
+      const int v = s_run[w * El1 + e];
+      s_run[w * El1 + e] = run;
+      run += v;
+    }
+  }
+  __syncthreads();
+
+  // placement: this warp's pairs in (token, slot) order, 32 at a time
+  const int gw0 = warp * kTokensPerWarp;
+  for (int r = 0; r < K; ++r) {
+    const int pidx = r * 32 + lane;
+    const int tl = pidx / K, k = pidx - tl * K;
+    const int key = mykeys[pidx];
+    const unsigned peers = __match_any_sync(0xffffffffu, key);
+    const int gg = gw0 + tl;
+    if (key >= 0) {
+      const int row = s_run[warp * El1 + key] + __popc(peers & lanemask_lt());
+      p.pos[static_cast<size_t>(gg) * K + k] = row;
+      p.row_token[row] = gg;
+      p.row_k[row] = k;
+      p.row_w[row] = mywt[pidx];
+    } else if (gg < T) {
+      p.pos[static_cast<size_t>(gg) * K + k] = -1;
+    }
+    __syncwarp();
+    if (key >= 0 && (31 - __clz(peers)) == static_cast<int>(lane)) s_run[warp * El1 + key] += __popc(peers);
+    __syncwarp();
+  }
+  if (g < T && p.S) {
+    const int row = s_goff[p.El] + g;
+    p.row_token[row] = g;
+    p.row_k[row] = -1;
+    p.row_w[row] = 1.0f;
+  }
+  // tokens that receive nothing from this GPU get zeros (only possible without a shared
+  // expert)
+  if (!p.S) {
+    unsigned need0 = __ballot_sync(0xffffffffu, g < T && need == 0);
+    while (need0) {
+      const int src_lane = __ffs(need0) - 1;
+      need0 &= need0 - 1;
+      const int mm = __shfl_sync(0xffffffffu, m, src_lane);
+      const int tt = __shfl_sync(0xffffffffu, t, src_lane);
+      uint4* dst = reinterpret_cast<uint4*>(slabs.y[mm] + static_cast<size_t>(tt) * p.H);
+      for (int i = lane; i < p.H / 8; i += 32) dst[i] = make_uint4(0, 0, 0, 0);
+    }
+  }
 }
 
 // 4. copy routed rows (FP8 codes and their per-128 scales) into expert order.
