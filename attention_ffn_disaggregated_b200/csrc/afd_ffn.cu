@@ -18,6 +18,7 @@
 #include <cstring>
 #include <mutex>
 #include <new>
+#include <utility>
 
 #include "afd_ffn.h"
 #include "gemm.cuh"
@@ -58,6 +59,25 @@ EncodeTiledFn get_encode_fn() {
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// One kernel launch; with `pdl` the kernel may start while the previous kernel in the
+// stream is still running (programmatic stream serialisation) and waits for it on the
+// device (pdl_wait) before touching its results.
+template <typename... KArgs, typename... Args>
+static void launch(bool pdl, void (*kernel)(KArgs...), int grid, int block, size_t smem,
+                   cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 }  // namespace
 
 struct afd_ffn_plan_s {
@@ -69,7 +89,7 @@ struct afd_ffn_plan_s {
   size_t ws_bytes = 0;
   int32_t *slab_base, *info, *chunk_hist, *chunk_off, *group_count, *group_off, *mtile_off;
   int tiling = 0;  // 0 = default (1); 2 = block-scale W13
-  int32_t *tok_mt, *tok_need, *pos, *row_token, *row_k;
+  int32_t *tok_mt, *tok_need, *pos, *row_token, *row_mt, *row_k;
   float* g_ws;        // split-K W13: fp32 sums [g_rows][2I], zero between calls
   int g_rows = 0;
   int* g_cnt;         // split-K W13: per (tile, quadrant) counters [num_sms][4]
@@ -88,6 +108,11 @@ struct afd_ffn_plan_s {
   unsigned long long wait_limit_ns = 1000000000ull;
   int inject_stall = 0;
   size_t scatter_smem = 0;
+  // combine destinations: the plan's own accumulators (slab m at acc + m*cap*H), or the
+  // caller's (afd_ffn_set_combine_targets; the layer then stops after W2)
+  AccTable own_acc;
+  AccTable ext_acc;
+  bool external_acc = false;
 };
 
 extern "C" {
@@ -110,7 +135,7 @@ const char* afd_status_string(afd_status_t s) {
 // tiling adds the activation factor images
 int32_t afd_ffn_kernels_per_layer(afd_ffn_plan_t P) {
   if (!P) return -1;
-  return (P->num_chunks <= kSmallRouteChunks ? 5 : 6) + (P->tiling == 2 ? 1 : 0);
+  return (P->num_chunks <= kSmallRouteChunks ? 5 : 6) + (P->tiling == 2 ? 1 : 0) - (P->external_acc ? 1 : 0);
 }
 
 afd_status_t afd_ffn_check_config(const afd_ffn_config_t* c) {
@@ -236,6 +261,7 @@ afd_status_t afd_ffn_plan(const afd_ffn_config_t* cfg, const afd_ffn_weights_t* 
   const size_t o_tok_need = take(sizeof(int32_t) * P->Tmax, 16);
   const size_t o_pos = take(sizeof(int32_t) * static_cast<size_t>(P->Tmax) * K, 16);
   const size_t o_row_token = take(sizeof(int32_t) * P->rpad, 16);
+  const size_t o_row_mt = take(sizeof(int32_t) * P->rpad, 16);
   const size_t o_row_k = take(sizeof(int32_t) * P->rpad, 16);
   const size_t o_row_w = take(sizeof(float) * P->rpad, 16);
   const size_t o_a_perm = take(static_cast<size_t>(P->rpad) * H, 1024);
@@ -275,6 +301,7 @@ afd_status_t afd_ffn_plan(const afd_ffn_config_t* cfg, const afd_ffn_weights_t* 
   P->tok_need = reinterpret_cast<int32_t*>(b + o_tok_need);
   P->pos = reinterpret_cast<int32_t*>(b + o_pos);
   P->row_token = reinterpret_cast<int32_t*>(b + o_row_token);
+  P->row_mt = reinterpret_cast<int32_t*>(b + o_row_mt);
   P->row_k = reinterpret_cast<int32_t*>(b + o_row_k);
   P->row_w = reinterpret_cast<float*>(b + o_row_w);
   P->a_perm = b + o_a_perm;
@@ -282,6 +309,9 @@ afd_status_t afd_ffn_plan(const afd_ffn_config_t* cfg, const afd_ffn_weights_t* 
   P->hq = b + o_hq;
   P->sh_t = reinterpret_cast<float*>(b + o_sh_t);
   P->acc = reinterpret_cast<float*>(b + o_acc);
+  memset(&P->own_acc, 0, sizeof(P->own_acc));
+  for (int m = 0; m < cfg->num_slabs; ++m)
+    P->own_acc.a[m] = P->acc + static_cast<size_t>(m) * cfg->slab_capacity * H;
   P->g_ws = reinterpret_cast<float*>(b + o_g_ws);
   P->g_cnt = reinterpret_cast<int*>(b + o_g_cnt);
   P->mx_sfa = b + o_mx_sfa;
@@ -377,6 +407,8 @@ static void fill_route_params(afd_ffn_plan_t P, const int32_t* d_counts, RoutePa
   rp.tok_need = P->tok_need;
   rp.pos = P->pos;
   rp.row_token = P->row_token;
+  rp.row_mt = P->row_mt;
+  rp.zero_y = P->external_acc ? 0 : 1;
   rp.row_k = P->row_k;
   rp.row_w = P->row_w;
   rp.a_perm = P->a_perm;
@@ -417,7 +449,8 @@ static void fill_gemm_params(afd_ffn_plan_t P, int epi, GemmParams& gp) {
     gp.w_scale = P->w.w2_scale;
     gp.ws_rows = c.hidden / 128;
     gp.row_w = P->row_w;
-    gp.acc = P->acc;
+    gp.row_mt = P->row_mt;
+    gp.acc = P->external_acc ? P->ext_acc : P->own_acc;
     gp.slice_first = P->w2_slice_first;
     gp.split_ok = 1;
   }
@@ -474,7 +507,20 @@ afd_status_t afd_ffn_layer(afd_ffn_plan_t P, const afd_slab_t* slabs, const int3
     route_scatter_kernel<<<P->num_chunks, kRouteThreads, P->scatter_smem, stream>>>(rp, tab);
   }
   if (tm) cudaEventRecord(P->ev[3], stream);
-  gather_rows_kernel<<<P->num_sms * 8, kRouteThreads, 0, stream>>>(rp, tab);
+  // one warp per token (gather) and per (token, 256 columns) (finalisation), grids no
+  // larger than the plan's capacity needs, so that small plans do not launch idle blocks
+  const int warps_per_block = kRouteThreads / 32;
+  const int gather_grid = std::max(1, std::min(P->num_sms * 8, (P->Tmax + warps_per_block - 1) / warps_per_block));
+  const int64_t fin_items = static_cast<int64_t>(P->Tmax) * (c.hidden / 256);
+  const int fin_grid = static_cast<int>(std::max<int64_t>(
+      1, std::min<int64_t>(P->num_sms * 4, (fin_items + warps_per_block - 1) / warps_per_block)));
+  // Small plans (one routing chunk) chain the kernels after the routing with programmatic
+  // dependent launch: each starts, sets itself up and waits on the device while its
+  // predecessor drains, instead of paying a launch gap at every step (at a few tokens the
+  // steps are a few microseconds each). Large plans launch in plain stream order: there
+  // the early GEMM blocks would hold SMs the gather still needs.
+  const bool pdl = P->num_chunks <= kSmallRouteChunks && !tm;
+  launch(pdl, gather_rows_kernel, gather_grid, kRouteThreads, 0, stream, rp, tab);
   if (tm) cudaEventRecord(P->ev[4], stream);
   const int grid = P->num_sms;
   if (mx) {
@@ -482,17 +528,19 @@ afd_status_t afd_ffn_layer(afd_ffn_plan_t P, const afd_slab_t* slabs, const int3
     // W13 stage time includes the image kernel)
     mx_act_sf_kernel<<<P->num_sms * 4, 128, 0, stream>>>(P->mtile_off, P->group_off, P->G, P->sa_t,
                                                          P->rpad, c.hidden / 128, P->mx_sfa, P->status);
-    w13_mx_kernel<<<grid, kGemmThreads, mx_smem_bytes(), stream>>>(g13, P->tm_a13, P->tm_w13,
-                                                                  MxArgs{P->mx_sfa, P->mx_sfb});
+    launch(pdl, w13_mx_kernel, grid, kGemmThreads, mx_smem_bytes(), stream, g13, P->tm_a13, P->tm_w13,
+           MxArgs{P->mx_sfa, P->mx_sfb});
   } else {
-    grouped_gemm_kernel<EPI_SWIGLU><<<grid, kGemmThreads, gemm_smem_bytes<EPI_SWIGLU>(), stream>>>(
-        g13, P->tm_a13, P->tm_w13);
+    launch(pdl, grouped_gemm_kernel<EPI_SWIGLU>, grid, kGemmThreads, gemm_smem_bytes<EPI_SWIGLU>(), stream,
+           g13, P->tm_a13, P->tm_w13);
   }
   if (tm) cudaEventRecord(P->ev[5], stream);
-  grouped_gemm_kernel<EPI_COMBINE><<<grid, kGemmThreads, gemm_smem_bytes<EPI_COMBINE>(), stream>>>(
-      g2, P->tm_a2, P->tm_w2);
+  launch(pdl, grouped_gemm_kernel<EPI_COMBINE>, grid, kGemmThreads, gemm_smem_bytes<EPI_COMBINE>(), stream,
+         g2, P->tm_a2, P->tm_w2);
   if (tm) cudaEventRecord(P->ev[6], stream);
-  combine_finalize_kernel<<<P->num_sms * 4, 256, 0, stream>>>(P->info, P->tok_mt, P->acc, c.hidden, ytab);
+  if (!P->external_acc)
+    launch(pdl, combine_finalize_kernel, fin_grid, 256, 0, stream, static_cast<const int32_t*>(P->info),
+           static_cast<const int32_t*>(P->tok_mt), P->own_acc, c.hidden, ytab);
   if (tm) cudaEventRecord(P->ev[7], stream);
   P->ev_valid = tm;
   if (cudaGetLastError() != cudaSuccess) return AFD_ERR_CUDA;
@@ -636,6 +684,57 @@ afd_status_t afd_ffn_inject_stall(afd_ffn_plan_t P, int32_t enable) {
   return AFD_OK;
 }
 
+afd_status_t afd_ffn_set_combine_targets(afd_ffn_plan_t P, float* const* acc_per_slab) {
+  if (!P) return AFD_ERR_INVALID_ARGUMENT;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev != P->device) return AFD_ERR_INVALID_ARGUMENT;
+  if (!acc_per_slab) {
+    P->external_acc = false;
+    return AFD_OK;
+  }
+  AccTable t;
+  memset(&t, 0, sizeof(t));
+  for (int m = 0; m < P->cfg.num_slabs; ++m) {
+    if (!acc_per_slab[m] || !aligned(acc_per_slab[m], 16)) return AFD_ERR_INVALID_ARGUMENT;
+    t.a[m] = acc_per_slab[m];
+  }
+  P->ext_acc = t;
+  P->external_acc = true;
+  return AFD_OK;
+}
+
+afd_status_t afd_combine_finalize(const afd_slab_t* slabs, int32_t num_slabs, int32_t slab_capacity,
+                                  int32_t hidden, const int32_t* d_counts, float* const* acc_per_slab,
+                                  afd_stream_t stream_) {
+  if (!slabs || !d_counts || !acc_per_slab) return AFD_ERR_INVALID_ARGUMENT;
+  if (num_slabs < 1 || num_slabs > AFD_MAX_SLABS || slab_capacity < 1 || slab_capacity > (1 << 24) - 1 ||
+      hidden < 256 || hidden % 256)
+    return AFD_ERR_INVALID_ARGUMENT;
+  AccTable acc;
+  YTable ytab;
+  memset(&acc, 0, sizeof(acc));
+  memset(&ytab, 0, sizeof(ytab));
+  for (int m = 0; m < num_slabs; ++m) {
+    if (!slabs[m].y || !aligned(slabs[m].y, 16) || !acc_per_slab[m] || !aligned(acc_per_slab[m], 16))
+      return AFD_ERR_INVALID_ARGUMENT;
+    acc.a[m] = acc_per_slab[m];
+    ytab.y[m] = static_cast<__nv_bfloat16*>(slabs[m].y);
+  }
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  // one warp per (token, 256 columns): enough blocks per slab to cover its capacity,
+  // at most a few waves of the GPU over all slabs
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return AFD_ERR_CUDA;
+  const int64_t items = static_cast<int64_t>(slab_capacity) * (hidden / 256);
+  const int per_slab = static_cast<int>(std::max<int64_t>(
+      1, std::min<int64_t>((sms * 4 + num_slabs - 1) / num_slabs, (items + 7) / 8)));
+  combine_finalize_slabs_kernel<<<dim3(per_slab, num_slabs), 256, 0, stream>>>(d_counts, slab_capacity, hidden,
+                                                                               acc, ytab);
+  if (cudaGetLastError() != cudaSuccess) return AFD_ERR_CUDA;
+  return AFD_OK;
+}
+
 }  // extern "C"
 
 // ------------------------------------------------------------------------------------
@@ -754,6 +853,7 @@ extern "C" afd_status_t afd_ffn_route_noalloc(const afd_ffn_config_t* cfg, const
   rp.row_w = d_row_weight;
   rp.status = d_status;
   rp.tiling = -1;           // routing only: d_sizes[3] = 0
+  rp.zero_y = 1;
   // every scratch region is fully written before it is read; only the status starts at 0
   if (cudaMemsetAsync(d_status, 0, sizeof(int32_t), stream) != cudaSuccess) return AFD_ERR_CUDA;
   const size_t scatter_smem = scatter_smem_bytes(El1, c.top_k);

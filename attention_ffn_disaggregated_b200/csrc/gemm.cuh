@@ -70,6 +70,12 @@ struct YTable {
   __nv_bfloat16* y[AFD_MAX_SLABS];
 };
 
+// Destination of the combine: token t of slab m adds into a[m] + t*H (the plan's own
+// accumulators, or buffers of the tokens' owners, possibly on other GPUs).
+struct AccTable {
+  float* a[AFD_MAX_SLABS];
+};
+
 struct GemmParams {
   const int32_t* info;        // [0] tokens, [1] rows, [2] m-tiles of this call
   const int32_t* group_off;   // [G+1] first row of each group
@@ -89,8 +95,9 @@ struct GemmParams {
   float* sh_t;                // [I/128][rpad]
   // COMBINE epilogue inputs/outputs
   const int32_t* row_token;
+  const int32_t* row_mt;      // (slab << 24) | row of each routed row's token
   const float* row_w;
-  float* acc;                 // [Tmax][H] fp32, zero between calls
+  AccTable acc;               // per slab: fp32 [cap][H], zero between calls
   // split-K for gate/up launches whose tiles fill less than half of the grid: the K blocks
   // of a tile are shared out among several CTAs, whose partial sums go to the fp32 workspace g_ws [g_rows][2I], and the CTA whose
   // partial completes a tile's 32-row quadrant (g_cnt) finishes SwiGLU + requantisation
@@ -262,6 +269,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     S.abort_flag = 0;
     fence_mbar_init();
   }
+  // everything above is local set-up; the tile schedule and the operands come from the
+  // previous kernels
+  pdl_trigger();
+  pdl_wait();
   for (int i = threadIdx.x; i <= p.G; i += blockDim.x) S.mtile[i] = p.mtile_off[i];
   if (warp == 1) {
     tmem_alloc(&S.tmem_base, kTmemCols);
@@ -437,6 +448,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       const float* ws0 = S.wring[wslot][EPI == EPI_SWIGLU ? 0 : half];
       const float* ws1 = S.wring[wslot][EPI == EPI_SWIGLU ? 1 : half];
+      // COMBINE: the row's destination and top-K weight, fetched before the K loop
+      int dst_mt = -1;
+      float wgt = 0.f;
+      if (EPI == EPI_COMBINE && valid) {
+        dst_mt = p.row_mt[grow];
+        wgt = p.row_w[grow];
+      }
       // acc[j] holds columns (2j, 2j+1) of this thread's 128: [0,32) from the first
       // 64-column group, [32,64) from the second
       float2 acc[64];
@@ -564,12 +582,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         // and issue their rows; before a buffer is refilled, the lanes that issued from it
         // last wait until the bulk engine has read it.
         const int col0 = c.nt * kBN + half * 128;
-        int g = -1;
-        float wgt = 0.f;
-        if (valid) {
-          g = p.row_token[grow];
-          wgt = p.row_w[grow];
-        }
+        float* dst = nullptr;
+        if (dst_mt >= 0)
+          dst = p.acc.a[dst_mt >> 24] + static_cast<size_t>(dst_mt & 0xFFFFFF) * p.H + col0;
         uint8_t* wst = stg + ew * kStgWarpBytes;
 #pragma unroll
         for (int r8 = 0; r8 < 4; ++r8) {
@@ -584,7 +599,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               *reinterpret_cast<float4*>(row + 4 * i) = make_float4(a.x * wgt, a.y * wgt, bb.x * wgt, bb.y * wgt);
             }
             fence_proxy_async_shared();
-            if (g >= 0) bulk_reduce_add_f32(p.acc + static_cast<size_t>(g) * p.H + col0, row, 512, pol_acc);
+            if (dst) bulk_reduce_add_f32(dst, row, 512, pol_acc);
             bulk_commit();
           }
         }
@@ -609,8 +624,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 // independent requests, not a chain of them).
 __global__ void __launch_bounds__(256) combine_finalize_kernel(const int32_t* __restrict__ info,
                                                                const int32_t* __restrict__ tok_mt,
-                                                               float* __restrict__ acc, int H,
+                                                               const __grid_constant__ AccTable acc, int H,
                                                                const __grid_constant__ YTable ytab) {
+  pdl_trigger();
+  pdl_wait();
   const int T = info[0];
   const int lane = threadIdx.x & 31;
   const int nseg = H / 256;                 // H is a multiple of 256
@@ -621,7 +638,38 @@ __global__ void __launch_bounds__(256) combine_finalize_kernel(const int32_t* __
     const int c = (it - g * nseg) * 256 + lane * 8;
     const int mt = tok_mt[g];
     const int m = mt >> 24, t = mt & 0xFFFFFF;
-    float* row = acc + static_cast<size_t>(g) * H;
+    float* row = acc.a[m] + static_cast<size_t>(t) * H;
+    __nv_bfloat16* y = ytab.y[m] + static_cast<size_t>(t) * H;
+    const float4 a = __ldcg(reinterpret_cast<const float4*>(row + c));
+    const float4 b = __ldcg(reinterpret_cast<const float4*>(row + c + 4));
+    uint4 o;
+    o.x = pack_bf16x2(a.x, a.y);
+    o.y = pack_bf16x2(a.z, a.w);
+    o.z = pack_bf16x2(b.x, b.y);
+    o.w = pack_bf16x2(b.z, b.w);
+    *reinterpret_cast<uint4*>(y + c) = o;
+    __stcg(reinterpret_cast<float4*>(row + c), make_float4(0.f, 0.f, 0.f, 0.f));
+    __stcg(reinterpret_cast<float4*>(row + c + 4), make_float4(0.f, 0.f, 0.f, 0.f));
+  }
+}
+
+// Expert-parallel return path, on the owner of the slabs: once every FFN GPU has added
+// its partial rows, token t < n_m of slab m becomes bf16 in y[m] and its accumulator row
+// is cleared. One warp per (slab, token, 256-column segment); blockIdx.y = slab.
+__global__ void __launch_bounds__(256) combine_finalize_slabs_kernel(const int32_t* __restrict__ counts,
+                                                                     int cap, int H,
+                                                                     const __grid_constant__ AccTable acc,
+                                                                     const __grid_constant__ YTable ytab) {
+  const int m = blockIdx.y;
+  const int n = min(max(counts[m], 0), cap);
+  const int lane = threadIdx.x & 31;
+  const int nseg = H / 256;
+  const int items = n * nseg;
+  const int nwarps = (gridDim.x * blockDim.x) >> 5;
+  for (int it = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; it < items; it += nwarps) {
+    const int t = it / nseg;
+    const int c = (it - t * nseg) * 256 + lane * 8;
+    float* row = acc.a[m] + static_cast<size_t>(t) * H;
     __nv_bfloat16* y = ytab.y[m] + static_cast<size_t>(t) * H;
     const float4 a = __ldcg(reinterpret_cast<const float4*>(row + c));
     const float4 b = __ldcg(reinterpret_cast<const float4*>(row + c + 4));

@@ -133,6 +133,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     S.abort_flag = 0;
     fence_mbar_init();
   }
+  // everything above is local set-up; the tile schedule and the operands come from the
+  // previous kernels
+  pdl_trigger();
+  pdl_wait();
   for (int i = threadIdx.x; i <= p.G; i += blockDim.x) S.mtile[i] = p.mtile_off[i];
   if (warp == 1) {
     tmem_alloc(&S.tmem_base, kTmemCols);

@@ -22,6 +22,15 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
+// Programmatic dependent launch. A kernel launched with programmatic stream serialisation
+// may start while the previous kernel in the stream is still running: it waits here
+// before its first access to that kernel's results (the wait returns once the previous
+// grid has completed and its memory is visible; without the launch attribute it returns
+// at once). The trigger lets the next kernel's blocks be scheduled as soon as every block
+// of this grid has issued it or exited.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ uint32_t lane_id() {
   uint32_t l;
   asm volatile("mov.u32 %0, %%laneid;" : "=r"(l));

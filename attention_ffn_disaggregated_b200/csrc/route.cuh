@@ -45,11 +45,13 @@ struct RouteParams {
   int32_t* tok_need;      // [Tmax] contributions this GPU adds to the token
   int32_t* pos;           // [Tmax*K]
   int32_t* row_token;     // [rpad]
+  int32_t* row_mt;        // [rpad] (slab << 24) | row of the row's token (may be null)
   int32_t* row_k;         // [rpad]
   float* row_w;           // [rpad]
   uint8_t* a_perm;        // [rpad][H]
   float* sa_t;            // [H/128][rpad]
   int* status;
+  int zero_y;             // zero the slab rows of tokens that receive nothing from this GPU
 };
 
 // Slab-major prefix of the valid row counts, clamped to [0, cap].
@@ -299,6 +301,10 @@ __device__ __forceinline__ void route_scatter_chunk(const RouteParams& p, const 
       p.row_token[row] = gg;
       p.row_k[row] = k;
       p.row_w[row] = mywt[pidx];
+      if (p.row_mt) {
+        const int mm = find_slab(s_base, p.M, gg);
+        p.row_mt[row] = (mm << 24) | (gg - s_base[mm]);
+      }
     } else {
       const int gg = gw0 + tl;
       if (gg < T) p.pos[static_cast<size_t>(gg) * K + k] = -1;
@@ -311,12 +317,13 @@ __device__ __forceinline__ void route_scatter_chunk(const RouteParams& p, const 
   if (g < T && p.S) {
     const int row = p.group_off[p.El] + g;
     p.row_token[row] = g;
+    if (p.row_mt) p.row_mt[row] = (m << 24) | t;
     p.row_k[row] = -1;
     p.row_w[row] = 1.0f;
   }
   // tokens that receive nothing from this GPU get zeros (only possible without a shared
   // expert); everything else is written by the down-projection's combine
-  if (!p.S) {
+  if (!p.S && p.zero_y) {
     unsigned need0 = __ballot_sync(0xffffffffu, g < T && p.tok_need[g] == 0);
     while (need0) {
       const int src_lane = __ffs(need0) - 1;
@@ -480,6 +487,10 @@ __global__ void __launch_bounds__(kRouteThreads) route_small_kernel(
       p.row_token[row] = gg;
       p.row_k[row] = k;
       p.row_w[row] = mywt[pidx];
+      if (p.row_mt) {
+        const int mm = find_slab(s_base, p.M, gg);
+        p.row_mt[row] = (mm << 24) | (gg - s_base[mm]);
+      }
     } else if (gg < T) {
       p.pos[static_cast<size_t>(gg) * K + k] = -1;
     }
@@ -490,12 +501,13 @@ __global__ void __launch_bounds__(kRouteThreads) route_small_kernel(
   if (g < T && p.S) {
     const int row = s_goff[p.El] + g;
     p.row_token[row] = g;
+    if (p.row_mt) p.row_mt[row] = (m << 24) | t;
     p.row_k[row] = -1;
     p.row_w[row] = 1.0f;
   }
   // tokens that receive nothing from this GPU get zeros (only possible without a shared
   // expert)
-  if (!p.S) {
+  if (!p.S && p.zero_y) {
     unsigned need0 = __ballot_sync(0xffffffffu, g < T && need == 0);
     while (need0) {
       const int src_lane = __ffs(need0) - 1;
@@ -515,6 +527,8 @@ __global__ void __launch_bounds__(kRouteThreads) route_small_kernel(
 // that a GEMM tile reads one block's scales for 32 consecutive rows with one load.
 __global__ void __launch_bounds__(kRouteThreads) gather_rows_kernel(
     const __grid_constant__ RouteParams p, const __grid_constant__ SlabTable slabs) {
+  pdl_trigger();
+  pdl_wait();
   const int T = p.info[0];
   const int K = p.K;
   const int lane = threadIdx.x & 31;

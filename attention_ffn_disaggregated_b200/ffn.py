@@ -90,6 +90,8 @@ def lib() -> ctypes.CDLL:
         "afd_ffn_set_tiling": (c_int32, [P, c_int32]),
         "afd_ffn_get_tiling": (c_int32, [P, P, POINTER(c_int32)]),
         "afd_ffn_kernels_per_layer": (c_int32, [P]),
+        "afd_ffn_set_combine_targets": (c_int32, [P, P]),
+        "afd_combine_finalize": (c_int32, [POINTER(SlabDesc), c_int32, c_int32, c_int32, P, P, P]),
         "afd_ffn_route_noalloc": (c_int32, [POINTER(Config), POINTER(SlabDesc), P, P, P, P, P, P, P, P,
                                             P, P]),
         "afd_status_string": (c_char_p, [c_int32]),
@@ -261,6 +263,46 @@ class FfnLayer:
 
     def inject_stall(self, enable: bool = True):
         lib().afd_ffn_inject_stall(self.plan, 1 if enable else 0)
+
+    def set_combine_targets(self, accs: Optional[Sequence]):
+        """Expert-parallel return path: the down projection adds each token's weighted rows
+        into accs[m] (fp32 [capacity, hidden] per received slab, possibly tensors that view
+        another GPU's memory) and the call stops after it; None restores the plan's own
+        accumulators and the bf16 slab outputs. The owner finishes with combine_finalize."""
+        if accs is None:
+            rc = lib().afd_ffn_set_combine_targets(self.plan, None)
+        else:
+            if len(accs) != self.num_slabs:
+                raise ValueError("expected %d accumulators" % self.num_slabs)
+            cap, H = self.slab_capacity, self.shape.hidden
+            for a in accs:
+                if str(a.dtype) != "torch.float32":
+                    raise ValueError("accumulators must be float32")
+                if tuple(a.shape) != (cap, H):
+                    raise ValueError(f"accumulator shape {tuple(a.shape)} != {(cap, H)}")
+            table = (c_void_p * self.num_slabs)(*[_ptr(a, "accumulator") for a in accs])
+            self._targets = accs            # the caller's buffers stay referenced while in use
+            rc = lib().afd_ffn_set_combine_targets(self.plan, table)
+        if rc != AFD_OK:
+            raise AfdError(rc, "afd_ffn_set_combine_targets")
+
+
+def combine_finalize(slabs: Sequence, counts, accs: Sequence, stream=None) -> None:
+    """Owner side of the expert-parallel return path: after every FFN GPU's partial rows
+    have been added into accs (fp32 [capacity, hidden] per slab), write y[m][t] =
+    bf16(accs[m][t]) for t < counts[m] and clear those accumulator rows."""
+    M = len(slabs)
+    if len(accs) != M:
+        raise ValueError("one accumulator per slab")
+    cap, H = accs[0].shape
+    descs = (SlabDesc * M)()
+    for i, s in enumerate(slabs):
+        descs[i] = SlabDesc(None, None, None, None, _ptr(s.y, "y"))
+    table = (c_void_p * M)(*[_ptr(a, "accumulator") for a in accs])
+    rc = lib().afd_combine_finalize(descs, M, int(cap), int(H), c_void_p(_ptr(counts, "counts")), table,
+                                    c_void_p(_stream_handle(stream)))
+    if rc != AFD_OK:
+        raise AfdError(rc, "afd_combine_finalize")
 
 
 def kernels_per_layer(layer: "FfnLayer") -> int:

@@ -297,9 +297,44 @@ AFD_API afd_status_t afd_ffn_route_noalloc(const afd_ffn_config_t* cfg, const af
                                            float* d_row_weight, int32_t* d_pos, int32_t* d_status,
                                            afd_stream_t stream);
 
+/*
+ * Expert-parallel return path. With the experts sharded over several FFN GPUs, each one
+ * computes a partial output for every token it received, and a token's result is the sum
+ * of the partials of all FFN GPUs, pushed back to the attention rank that owns the token
+ * (FastAFD, "Methodology / System Design", item 3, push-back M2N; items 2-3 for the
+ * receive buffers that the attention ranks write into).
+ *
+ * afd_ffn_set_combine_targets: from the next afd_ffn_layer call on, the down projection
+ * of this plan adds each token's weighted expert rows (fp32, one reduction per element)
+ * into acc_per_slab[m] + t * hidden for token t of received slab m, instead of into the
+ * plan's own accumulators, and the layer call stops there: no finalisation launch, and
+ * no slab y row is written. acc_per_slab: HOST array of num_slabs device pointers to fp32
+ * [slab_capacity][hidden] buffers, 16-byte aligned; they may be other GPUs' memory mapped
+ * into this device's address space (peer pointers), and several plans, on this or other
+ * GPUs, may add into the same buffers at the same time. The buffers must hold zeros where
+ * rows will be added before the first such call (afd_combine_finalize leaves them zero).
+ * NULL restores the plan's own accumulators and the bf16 slab outputs. Copies the table
+ * to the device (synchronous). AFD_ERR_INVALID_ARGUMENT for a NULL plan, a NULL or
+ * misaligned entry, or a current device other than the plan's.
+ *
+ * afd_combine_finalize: on the GPU of the owning attention rank, once every FFN GPU's
+ * additions have completed: for each of num_slabs slabs and t < counts[m], writes
+ * y[m][t] = bf16(acc_per_slab[m][t]) (round to nearest even) and clears that accumulator
+ * row. slabs: host array (only y is used); d_counts: device int32 [num_slabs], clamped
+ * to [0, slab_capacity] on the device; acc_per_slab: host array of device pointers as
+ * above. Enqueued on `stream`, never synchronises. AFD_ERR_INVALID_ARGUMENT for NULL or
+ * misaligned pointers or sizes out of range (num_slabs 1..AFD_MAX_SLABS, hidden a positive
+ * multiple of 256), AFD_ERR_CUDA if the launch fails.
+ */
+AFD_API afd_status_t afd_ffn_set_combine_targets(afd_ffn_plan_t plan, float* const* acc_per_slab);
+AFD_API afd_status_t afd_combine_finalize(const afd_slab_t* slabs, int32_t num_slabs, int32_t slab_capacity,
+                                          int32_t hidden, const int32_t* d_counts,
+                                          float* const* acc_per_slab, afd_stream_t stream);
+
 /* Number of this library's kernel launches one afd_ffn_layer call of this plan makes with
  * its current tiling: 6, or 5 when num_slabs * slab_capacity <= 256 (the routing runs in
- * one block), one more with tiling 2. -1 for NULL. */
+ * one block), one more with tiling 2, one fewer with combine targets set (no
+ * finalisation). -1 for NULL. */
 AFD_API int32_t afd_ffn_kernels_per_layer(afd_ffn_plan_t plan);
 
 /* Human-readable name of a status code. */

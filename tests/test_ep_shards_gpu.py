@@ -51,3 +51,69 @@ def test_two_expert_shards_sum_to_the_full_layer(counts, cap, zipf):
     err = np.abs(total - ref).max(axis=1)
     # two bf16 roundings instead of one: the same row tolerance still holds comfortably
     assert np.all(err <= TOL_ROW_RMS * rms), float((err / rms).max())
+
+
+@pytest.mark.parametrize("counts,cap,zipf,shared_on_a", [
+    ([200, 37, 0, 129], 200, None, True),
+    ([96, 5], 128, 1.0, False),      # no shared expert: tokens that touch no held expert
+])
+def test_shards_add_into_the_owners_accumulators(counts, cap, zipf, shared_on_a):
+    """The return path fused into the down projection: both shards' plans add their weighted
+    expert rows straight into one set of per-slab fp32 accumulators (on an expert-parallel
+    pool these are the owning attention rank's buffers, reached through peer pointers), and
+    the owner's finalisation rounds each token's sum once to bf16 and clears the buffers.
+    Run twice, so that the second step starts from the cleared accumulators."""
+    import torch
+    from attention_ffn_disaggregated_b200 import FfnLayer, kernels_per_layer
+    from attention_ffn_disaggregated_b200.device import (gather_outputs, to_device_counts,
+                                                          to_device_slabs, to_device_weights)
+    from attention_ffn_disaggregated_b200.ffn import combine_finalize
+    from tests.helpers import compare_outputs
+
+    H, I, Eg, K = 512, 256, 16, 4
+    S = 1 if shared_on_a else 0
+    full = W.make_custom_inputs(W.LayerShape(H, I, Eg, 0, Eg, S, K), counts, cap, seed=43, zipf_s=zipf)
+    a = _shard(full, W.LayerShape(H, I, Eg, 0, 8, S, K), 0, 8, bool(S))
+    b = _shard(full, W.LayerShape(H, I, Eg, 8, 8, 0, K), 8, 16, False)
+    slabs = to_device_slabs(full)
+    cnt = to_device_counts(full)
+    accs = [torch.zeros((cap, H), dtype=torch.float32, device="cuda") for _ in counts]
+    layers = [FfnLayer(sh.shape, len(counts), cap, *to_device_weights(sh)) for sh in (a, b)]
+    for L in layers:
+        n0 = kernels_per_layer(L)
+        L.set_combine_targets(accs)
+        assert kernels_per_layer(L) == n0 - 1          # no finalisation launch
+    for step in range(2):
+        for s in slabs:
+            s.y.fill_(float("nan"))
+        for L in layers:
+            L(slabs, cnt)
+        # the plans write no slab output of their own
+        torch.cuda.synchronize()
+        assert all(bool(torch.isnan(s.y[:n].float()).all()) for s, n in zip(slabs, counts) if n)
+        combine_finalize(slabs, cnt, accs)
+        torch.cuda.synchronize()
+        y = gather_outputs(full, slabs)
+        # the oracle: each shard's partial on that shard's codes (the GPU's midpoint
+        # decisions taken over), added in float64
+        ref = 0.0
+        for L, shard in zip(layers, (a, b)):
+            assert L.status()[0] == 0
+            codes_g, scales_g = L.intermediate()
+            o = offn.ffn_layer(shard, keep_intermediates=True)
+            rows = np.arange(o["routing"].num_rows)
+            codes, _ = reconcile_codes(codes_g, scales_g, o["h32"], o["h_codes"], o["h_scales"], rows)
+            ref = ref + offn.down_and_combine(shard, o["routing"], codes, o["h_scales"])
+        compare_outputs(y, ref)
+        for acc, n in zip(accs, counts):
+            assert float(acc.abs().max()) == 0.0             # cleared for the next step
+    # targets removed: the plan writes its own bf16 partial again
+    layers[0].set_combine_targets(None)
+    for s in slabs:
+        s.y.fill_(float("nan"))
+    layers[0](slabs, cnt)
+    torch.cuda.synchronize()
+    compare_layer({"outs": [gather_outputs(a, slabs)], "routing": layers[0].routing(),
+                   "h_codes": layers[0].intermediate()[0], "h_scales": layers[0].intermediate()[1]}, a)
+    for L in layers:
+        L.close()
