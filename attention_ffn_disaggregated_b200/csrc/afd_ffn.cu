@@ -382,6 +382,7 @@ afd_status_t afd_ffn_get_info(afd_ffn_plan_t P, afd_ffn_plan_info_t* info) {
 
 static void fill_route_params(afd_ffn_plan_t P, const int32_t* d_counts, RouteParams& rp) {
   const afd_ffn_config_t& c = P->cfg;
+  memset(&rp, 0, sizeof(rp));
   rp.counts = d_counts;
   rp.M = c.num_slabs;
   rp.cap = c.slab_capacity;
@@ -409,6 +410,7 @@ static void fill_route_params(afd_ffn_plan_t P, const int32_t* d_counts, RoutePa
   rp.row_token = P->row_token;
   rp.row_mt = P->row_mt;
   rp.zero_y = P->external_acc ? 0 : 1;
+
   rp.row_k = P->row_k;
   rp.row_w = P->row_w;
   rp.a_perm = P->a_perm;
@@ -418,6 +420,7 @@ static void fill_route_params(afd_ffn_plan_t P, const int32_t* d_counts, RoutePa
 
 static void fill_gemm_params(afd_ffn_plan_t P, int epi, GemmParams& gp) {
   const afd_ffn_config_t& c = P->cfg;
+  const bool small = P->num_chunks <= kSmallRouteChunks;
   memset(&gp, 0, sizeof(gp));
   gp.info = P->info;
   gp.group_off = P->group_off;
@@ -434,6 +437,11 @@ static void fill_gemm_params(afd_ffn_plan_t P, int epi, GemmParams& gp) {
     gp.num_kb = c.hidden / 128;
     gp.sa_t = P->sa_t;
     gp.w_scale = P->w.w13_scale;
+    if (small && c.has_shared_expert) {
+      // the shared expert's W13 (every token's), prefetched while the gather runs
+      gp.pf_base = static_cast<const uint8_t*>(P->w.w13) + static_cast<size_t>(c.num_local_experts) * 2 * c.intermediate * c.hidden;
+      gp.pf_bytes = static_cast<unsigned long long>(2) * c.intermediate * c.hidden;
+    }
     gp.ws_rows = 2 * c.intermediate / 128;
     gp.hq = P->hq;
     gp.sh_t = P->sh_t;
@@ -447,6 +455,10 @@ static void fill_gemm_params(afd_ffn_plan_t P, int epi, GemmParams& gp) {
     gp.num_kb = c.intermediate / 128;
     gp.sa_t = P->sh_t;
     gp.w_scale = P->w.w2_scale;
+    if (small && c.has_shared_expert) {
+      gp.pf_base = static_cast<const uint8_t*>(P->w.w2) + static_cast<size_t>(c.num_local_experts) * c.hidden * c.intermediate;
+      gp.pf_bytes = static_cast<unsigned long long>(c.hidden) * c.intermediate;
+    }
     gp.ws_rows = c.hidden / 128;
     gp.row_w = P->row_w;
     gp.row_mt = P->row_mt;
@@ -501,7 +513,7 @@ afd_status_t afd_ffn_layer(afd_ffn_plan_t P, const afd_slab_t* slabs, const int3
     if (tm) cudaEventRecord(P->ev[2], stream);
   } else {
     // the routing scan runs in route_count's last block (its stage time reads as zero)
-    route_count_kernel<<<P->num_chunks, kRouteThreads, 0, stream>>>(rp, tab);
+    route_count_kernel<<<P->num_chunks, kRouteThreads, sizeof(int32_t) * kChunkTokens * c.top_k, stream>>>(rp, tab);
     if (tm) cudaEventRecord(P->ev[1], stream);
     if (tm) cudaEventRecord(P->ev[2], stream);
     route_scatter_kernel<<<P->num_chunks, kRouteThreads, P->scatter_smem, stream>>>(rp, tab);
@@ -857,7 +869,7 @@ extern "C" afd_status_t afd_ffn_route_noalloc(const afd_ffn_config_t* cfg, const
   // every scratch region is fully written before it is read; only the status starts at 0
   if (cudaMemsetAsync(d_status, 0, sizeof(int32_t), stream) != cudaSuccess) return AFD_ERR_CUDA;
   const size_t scatter_smem = scatter_smem_bytes(El1, c.top_k);
-  route_count_kernel<<<static_cast<int>(chunks), kRouteThreads, 0, stream>>>(rp, tab);
+  route_count_kernel<<<static_cast<int>(chunks), kRouteThreads, sizeof(int32_t) * kChunkTokens * c.top_k, stream>>>(rp, tab);
   route_scan_kernel<<<1, 1024, 0, stream>>>(rp);
   route_scatter_kernel<<<static_cast<int>(chunks), kRouteThreads, scatter_smem, stream>>>(rp, tab);
   if (cudaGetLastError() != cudaSuccess) return AFD_ERR_CUDA;

@@ -106,6 +106,11 @@ struct GemmParams {
   float* g_ws;
   int g_rows;
   int* g_cnt;                 // [grid][4], zero between calls
+  // weights every call of a small plan reads (the shared expert's), prefetched into L2 by
+  // the CTAs, spread over all of them, while the previous kernels still run; null when
+  // not used
+  const uint8_t* pf_base;
+  unsigned long long pf_bytes;
   int* status;
   unsigned long long wait_limit_ns;
   int inject_stall;
@@ -131,6 +136,7 @@ struct alignas(16) GemmSmem {
   int abort_flag;
   float amax[2][2][kTileM];
   int32_t mtile[AFD_MAX_GROUPS + 1];
+  int32_t goff[AFD_MAX_GROUPS + 1];   // first row of each group (tile decoding)
 };
 static_assert(sizeof(GemmSmem) % 16 == 0, "staging after GemmSmem must stay 16-byte aligned");
 
@@ -269,14 +275,32 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     S.abort_flag = 0;
     fence_mbar_init();
   }
-  // everything above is local set-up; the tile schedule and the operands come from the
-  // previous kernels
-  pdl_trigger();
-  pdl_wait();
-  for (int i = threadIdx.x; i <= p.G; i += blockDim.x) S.mtile[i] = p.mtile_off[i];
   if (warp == 1) {
     tmem_alloc(&S.tmem_base, kTmemCols);
     tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_a);
+    tma_prefetch_desc(&tm_b);
+  }
+  if (p.pf_bytes && warp == 2) {
+    // this CTA's share of the always-read weights, in 16-byte multiples, 32 KiB per request
+    const unsigned long long share = ((p.pf_bytes + gridDim.x - 1) / gridDim.x + 15ull) & ~15ull;
+    const unsigned long long lo = share * blockIdx.x;
+    const unsigned long long hi = lo + share < p.pf_bytes ? lo + share : p.pf_bytes;
+    for (unsigned long long o = lo + 32768ull * lane; o < hi; o += 32768ull * 32)
+      bulk_prefetch_l2(p.pf_base + o, static_cast<uint32_t>(hi - o < 32768ull ? hi - o : 32768ull));
+  }
+
+  // everything above is local set-up (a kernel launched early under programmatic
+  // dependent launch does it while its predecessor drains; no predecessor holds tensor
+  // memory on this SM, whose shared memory this kernel fills); the tile schedule and the
+  // operands come from the previous kernels
+  pdl_trigger();
+  pdl_wait();
+  for (int i = threadIdx.x; i <= p.G; i += blockDim.x) {
+    S.mtile[i] = p.mtile_off[i];
+    S.goff[i] = p.group_off[i];
   }
   tc_fence_before();
   __syncthreads();
@@ -298,8 +322,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kProducerRegs));
     if (warp == 0 && lane == 0) {
       // ---------------------------------------------------------------- TMA producer
-      tma_prefetch_desc(&tm_a);
-      tma_prefetch_desc(&tm_b);
       // A rows are re-read by every column tile of their m-tile. W13 weight blocks are
       // re-read by every m-tile of their expert; W2's stream past the L2-resident combine
       // accumulators, so they go first.
@@ -311,7 +333,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       for (int u = blockIdx.x; ok && u < total_units; u += gridDim.x) {
         const int tile = u / splits, sp = u - tile * splits;
         const int kb0 = sp * nkb / splits, kb1 = (sp + 1) * nkb / splits;
-        const TileCoord c = decode_tile(tile, p.n_tiles, p.slice_first, S.mtile, p.G, p.group_off);
+        const TileCoord c = decode_tile(tile, p.n_tiles, p.slice_first, S.mtile, p.G, S.goff);
         // B rows of this tile: [brow0, +128) and [brow1, +128)
         int brow0, brow1;
         if (EPI == EPI_SWIGLU) {
@@ -391,7 +413,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int j = 0;
       for (int u = blockIdx.x; u < total_units; u += gridDim.x, ++j) {
         const int tile = u / splits;
-        const TileCoord c = decode_tile(tile, p.n_tiles, p.slice_first, S.mtile, p.G, p.group_off);
+        const TileCoord c = decode_tile(tile, p.n_tiles, p.slice_first, S.mtile, p.G, S.goff);
         const int r0 = EPI == EPI_SWIGLU ? c.nt : 2 * c.nt;
         const int r1 = EPI == EPI_SWIGLU ? p.I / 128 + c.nt : 2 * c.nt + 1;
         const float* w0 = p.w_scale + (static_cast<size_t>(c.e) * p.ws_rows + r0) * nkb;
@@ -426,7 +448,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     for (int u = blockIdx.x; ok && u < total_units; u += gridDim.x, ++titer) {
       const int tile = u / splits, sp = u - tile * splits;
       const int kb0 = sp * nkb / splits, kb1 = (sp + 1) * nkb / splits;
-      const TileCoord c = decode_tile(tile, p.n_tiles, p.slice_first, S.mtile, p.G, p.group_off);
+      const TileCoord c = decode_tile(tile, p.n_tiles, p.slice_first, S.mtile, p.G, S.goff);
       const int grow = c.row0 + trow;
       const bool valid = trow < c.rows;
       int c0, c1;

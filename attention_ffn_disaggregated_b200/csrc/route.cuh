@@ -83,25 +83,23 @@ __device__ __forceinline__ int find_slab(const int32_t* s_base, int M, int g) {
   return lo;
 }
 
-// Classify the K slots of one token. Returns a mask of the slots that are valid and
-// local; `le[k]` receives the local group of slot k. Sets *bad for ids that are neither
-// -1 nor in [0, E_g), and for ids repeated from an earlier slot.
-__device__ __forceinline__ uint32_t classify_token(const int32_t* ids, int K, int e0, int El,
-                                                   int Eg, int* le, bool* bad) {
+// Classify the K slots of one token, in shared memory: keys[0..K) hold the token's ids on
+// entry and, on return, the local group of each slot (-1 if the slot is not used here).
+// Returns the mask of the slots that are valid and local. Sets *bad for ids that are
+// neither -1 nor in [0, E_g), and for ids repeated from an earlier slot. (No per-thread
+// arrays, so no local memory.)
+__device__ __forceinline__ uint32_t classify_keys(int32_t* keys, int K, int e0, int El, int Eg, bool* bad) {
   uint32_t mask = 0;
   for (int k = 0; k < K; ++k) {
-    const int id = ids[k];
-    le[k] = -1;
+    const int id = keys[k];
     if (id == -1) continue;
     if (id < 0 || id >= Eg) { *bad = true; continue; }
     bool dup = false;
-    for (int j = 0; j < k; ++j) dup |= (ids[j] == id);
+    for (int j = 0; j < k; ++j) dup |= (keys[j] == id);
     if (dup) { *bad = true; continue; }
-    if (id >= e0 && id < e0 + El) {
-      le[k] = id - e0;
-      mask |= 1u << k;
-    }
+    if (id >= e0 && id < e0 + El) mask |= 1u << k;
   }
+  for (int k = 0; k < K; ++k) keys[k] = (mask >> k & 1u) ? keys[k] - e0 : -1;
   return mask;
 }
 
@@ -183,24 +181,23 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(const __grid_constant_
 
 // 1 for one chunk of 256 tokens (thread = token): classification, histogram of the local
 // groups in shared memory, token bookkeeping; the histogram goes to chunk_hist[chunk].
-// Called by all threads of the block.
+// s_keys: shared memory [256][K] for the tokens' ids. Called by all threads of the block.
 __device__ __forceinline__ void route_count_chunk(const RouteParams& p, const SlabTable& slabs,
                                                   const int32_t* s_base, int T, int chunk,
-                                                  int32_t* s_hist) {
+                                                  int32_t* s_hist, int32_t* s_keys) {
   for (int e = threadIdx.x; e < p.El; e += blockDim.x) s_hist[e] = 0;
   __syncthreads();
   const int g = chunk * kChunkTokens + threadIdx.x;
   if (g < T) {
     const int m = find_slab(s_base, p.M, g);
     const int t = g - s_base[m];
-    int32_t ids[AFD_MAX_TOP_K];
-    int le[AFD_MAX_TOP_K];
+    int32_t* keys = s_keys + threadIdx.x * p.K;
     const int32_t* src = slabs.ids[m] + static_cast<size_t>(t) * p.K;
-    for (int k = 0; k < p.K; ++k) ids[k] = src[k];
+    for (int k = 0; k < p.K; ++k) keys[k] = src[k];
     bool bad = false;
-    uint32_t mask = classify_token(ids, p.K, p.e0, p.El, p.Eg, le, &bad);
+    const uint32_t mask = classify_keys(keys, p.K, p.e0, p.El, p.Eg, &bad);
     for (int k = 0; k < p.K; ++k)
-      if (mask >> k & 1u) atomicAdd(&s_hist[le[k]], 1);
+      if (mask >> k & 1u) atomicAdd(&s_hist[keys[k]], 1);
     p.tok_mt[g] = (m << 24) | t;
     p.tok_need[g] = __popc(mask) + p.S;
     if (bad) atomicOr(p.status, AFD_STATUS_BAD_ROUTING);
@@ -214,8 +211,10 @@ __device__ __forceinline__ void route_count_chunk(const RouteParams& p, const Sl
 // 1. per-chunk histogram of local groups; token bookkeeping. With p.scan_ticket set, the
 // block that finishes last also runs step 2 (every block publishes its histogram, fences,
 // then takes a ticket; the counter is returned to zero for the next call).
+// Dynamic shared memory: the ids of the chunk's tokens, [256][K] int32.
 __global__ void __launch_bounds__(kRouteThreads) route_count_kernel(
     const __grid_constant__ RouteParams p, const __grid_constant__ SlabTable slabs) {
+  extern __shared__ int32_t s_keys[];
   __shared__ int32_t s_base[AFD_MAX_SLABS + 1];
   __shared__ int32_t s_hist[AFD_MAX_GROUPS];
   load_slab_base(p, s_base);
@@ -224,7 +223,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_count_kernel(
     for (int m = threadIdx.x; m <= p.M; m += blockDim.x) p.slab_base[m] = s_base[m];
     if (threadIdx.x == 0) p.info[0] = T;
   }
-  route_count_chunk(p, slabs, s_base, T, blockIdx.x, s_hist);
+  route_count_chunk(p, slabs, s_base, T, blockIdx.x, s_hist, s_keys);
   if (!p.scan_ticket) return;
   __shared__ int s_last;
   __shared__ int s_warp[32];
@@ -257,20 +256,17 @@ __device__ __forceinline__ void route_scatter_chunk(const RouteParams& p, const 
   if (g < T) {
     m = find_slab(s_base, p.M, g);
     t = g - s_base[m];
-    int32_t ids[AFD_MAX_TOP_K];
-    int le[AFD_MAX_TOP_K];
     const int32_t* src = slabs.ids[m] + static_cast<size_t>(t) * K;
     const float* wsrc = slabs.w[m] + static_cast<size_t>(t) * K;
+    int32_t* keys = mykeys + lane * K;
     for (int k = 0; k < K; ++k) {
-      ids[k] = src[k];
+      keys[k] = src[k];
       mywt[lane * K + k] = wsrc[k];
     }
     bool bad = false;
-    classify_token(ids, K, p.e0, p.El, p.Eg, le, &bad);
-    for (int k = 0; k < K; ++k) {
-      mykeys[lane * K + k] = le[k];
-      if (le[k] >= 0) atomicAdd(&s_run[warp * El1 + le[k]], 1);
-    }
+    const uint32_t mask = classify_keys(keys, K, p.e0, p.El, p.Eg, &bad);
+    for (int k = 0; k < K; ++k)
+      if (mask >> k & 1u) atomicAdd(&s_run[warp * El1 + keys[k]], 1);
   } else {
     for (int k = 0; k < K; ++k) mykeys[lane * K + k] = -1;
   }
@@ -376,6 +372,8 @@ __global__ void __launch_bounds__(kRouteThreads) route_small_kernel(
   int32_t* s_key = s_dyn + kRouteWarps * El1;     // [warps][32*K]
   float* s_wt = reinterpret_cast<float*>(s_key + kRouteWarps * 32 * K);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // the gather may be scheduled now; it waits for this kernel's results on the device
+  pdl_trigger();
 
   // slab bases: one count per thread (M <= 128), clamped, block scan
   int n = 0;
@@ -408,20 +406,17 @@ __global__ void __launch_bounds__(kRouteThreads) route_small_kernel(
   if (g < T) {
     m = find_slab(s_base, p.M, g);
     t = g - s_base[m];
-    int32_t ids[AFD_MAX_TOP_K];
-    int le[AFD_MAX_TOP_K];
     const int32_t* src = slabs.ids[m] + static_cast<size_t>(t) * K;
     const float* wsrc = slabs.w[m] + static_cast<size_t>(t) * K;
+    int32_t* keys = mykeys + lane * K;
     for (int k = 0; k < K; ++k) {
-      ids[k] = src[k];
+      keys[k] = src[k];
       mywt[lane * K + k] = wsrc[k];
     }
     bool bad = false;
-    const uint32_t mask = classify_token(ids, K, p.e0, p.El, p.Eg, le, &bad);
-    for (int k = 0; k < K; ++k) {
-      mykeys[lane * K + k] = le[k];
-      if (le[k] >= 0) atomicAdd(&s_run[warp * El1 + le[k]], 1);
-    }
+    const uint32_t mask = classify_keys(keys, K, p.e0, p.El, p.Eg, &bad);
+    for (int k = 0; k < K; ++k)
+      if (mask >> k & 1u) atomicAdd(&s_run[warp * El1 + keys[k]], 1);
     need = __popc(mask) + p.S;
     p.tok_mt[g] = (m << 24) | t;
     p.tok_need[g] = need;
