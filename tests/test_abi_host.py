@@ -115,3 +115,29 @@ def test_binding_refuses_host_tensors():
     assert _ptr(None) is None
     with pytest.raises(ValueError, match="w13 must be a CUDA tensor"):
         _ptr(torch.zeros(16, dtype=torch.uint8), "w13")
+
+
+def test_return_path_entry_points_validate_arguments():
+    """afd_ffn_set_combine_targets and afd_combine_finalize refuse bad arguments before
+    touching a GPU (NULL plan or tables, misaligned or NULL buffers, sizes out of range)."""
+    L = ffn.lib()
+    assert L.afd_ffn_set_combine_targets(None, None) == 1
+    slabs = (ffn.SlabDesc * 2)()
+    for i in range(2):
+        slabs[i] = ffn.SlabDesc(None, None, None, None, 0x10000 + 0x1000 * i)
+    acc = (ctypes.c_void_p * 2)(0x20000, 0x30000)
+    counts = ctypes.c_void_p(0x40000)
+    fin = L.afd_combine_finalize
+    assert fin(None, 2, 8, 256, counts, acc, None) == 1                  # no slabs
+    assert fin(slabs, 2, 8, 256, None, acc, None) == 1                   # no counts
+    assert fin(slabs, 2, 8, 256, counts, None, None) == 1                # no accumulators
+    assert fin(slabs, 0, 8, 256, counts, acc, None) == 1                 # no slabs to finish
+    assert fin(slabs, 129, 8, 256, counts, acc, None) == 1               # above the slab limit
+    assert fin(slabs, 2, 0, 256, counts, acc, None) == 1                 # zero capacity
+    assert fin(slabs, 2, 8, 384, counts, acc, None) == 1                 # hidden not a multiple of 256
+    bad = (ctypes.c_void_p * 2)(0x20000, 0x30004)                        # misaligned accumulator
+    assert fin(slabs, 2, 8, 256, counts, bad, None) == 1
+    nul = (ctypes.c_void_p * 2)(0x20000, None)
+    assert fin(slabs, 2, 8, 256, counts, nul, None) == 1
+    slabs[1] = ffn.SlabDesc(None, None, None, None, 0x10008)              # misaligned output rows
+    assert fin(slabs, 2, 8, 256, counts, acc, None) == 1
