@@ -22,7 +22,15 @@
 //            512-byte row segment per operation, staged through shared memory), so the
 //            epilogue warps hand the reductions off and return to the next tile's partial
 //            products; combine_finalize_kernel then writes every token's sum as bf16 into
-//            its slab row and clears the accumulator.
+//            its slab row and clears the accumulator. The accumulator of token t of slab m
+//            is found through a per-slab pointer table (the plan's own buffers, or the
+//            tokens' owners' under expert parallelism).
+//
+// Small batches: when the tiles fill at most half of the grid, each tile's K blocks are
+// shared out among several CTAs (split-K); W13's splits meet in an fp32 workspace and the
+// last one finishes the tile, W2's partial sums are reduced into the accumulators like
+// whole tiles. Under programmatic dependent launch a CTA allocates TMEM and prefetches
+// its descriptors before waiting for the previous kernel.
 #pragma once
 
 #include "ptx.cuh"

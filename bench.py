@@ -103,15 +103,26 @@ KERNEL_SOURCES = {
 }
 
 
+def code_tokens(text: str) -> str:
+    """C/C++/CUDA source with comments removed and whitespace runs collapsed: what the
+    compiler sees, so that editing a comment does not change a kernel's record key."""
+    import re
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
 def source_hash(kernel: str = "") -> str:
-    """Hash of the files `kernel` is built from (of the whole CUDA tree without a name)."""
+    """Hash of the code (comments and layout ignored) of the files `kernel` is built from
+    (of the whole CUDA tree without a name)."""
     files = KERNEL_SOURCES.get(kernel)
     if files is None:
         files = [os.path.join(d, f) for d in (CSRC.rstrip("/"), "include")
                  for f in sorted(os.listdir(os.path.join(ROOT, d)))]
     h = hashlib.sha256()
     for f in files:
-        h.update(open(os.path.join(ROOT, f), "rb").read())
+        h.update(code_tokens(open(os.path.join(ROOT, f), encoding="utf-8").read()).encode())
+        h.update(b"\0")
     return h.hexdigest()[:16]
 
 
