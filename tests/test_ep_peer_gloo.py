@@ -1,13 +1,13 @@
 """The peer-memory EP exchange (attention_ffn_disaggregated_b200.ep.PeerEpExchange) on the
-CPU: gloo, world size 2, shared-memory tensors standing in for peer-mapped device memory.
+CPU: gloo, world sizes 2 and 4, shared-memory tensors standing in for peer-mapped device memory.
 
-Each rank owns two slabs of tokens (its attention side) and half of the experts (its FFN
-side; the shared expert on rank 0). Per step: every rank copies its slabs into both
-ranks' receive buffers, each FFN rank adds its partial rows for every received token
+Each rank owns two slabs of tokens (its attention side) and 1/world of the experts (its
+FFN side; the shared expert on rank 0); world sizes 2 and 4. Per step: every rank copies
+its slabs into every rank's receive buffers, each FFN rank adds its partial rows for every received token
 straight into the owning rank's fp32 accumulators (the ranks take turns here; on GPUs the
 down projection's reductions are atomic), and after a barrier each owner rounds its sums to
 bf16 and clears them. Checked on two consecutive steps: each owner's outputs are exactly
-the bf16 of the fp32 sum of both shards' partials, and within the row tolerance of the full
+the bf16 of the fp32 sum of all shards' partials, and within the row tolerance of the full
 layer with all experts on one GPU. The layer is played by the oracle (the kernels' side of
 this path, adding into shared accumulators, is tested on one GPU in
 tests/test_ep_shards_gpu.py).
@@ -16,6 +16,7 @@ import os
 import socket
 
 import numpy as np
+import pytest
 import torch
 import torch.distributed as dist
 import torch.multiprocessing as mp
@@ -24,7 +25,7 @@ import workloads as W
 
 FULL = W.LayerShape(256, 128, 8, 0, 8, 1, 3)
 CAP = 12
-COUNTS = {0: [7, 12], 1: [0, 5]}
+COUNTS = {0: [7, 12], 1: [0, 5], 2: [12, 1], 3: [3, 0]}
 
 
 def _free_port():
@@ -103,14 +104,15 @@ def _worker(rank, world, port, out_q):
         dist.destroy_process_group()
 
 
-def test_peer_exchange_adds_partials_into_the_owners_accumulators():
+@pytest.mark.parametrize("world", [2, 4])
+def test_peer_exchange_adds_partials_into_the_owners_accumulators(world):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    procs = [ctx.Process(target=_worker, args=(r, world, port, q)) for r in range(world)]
     for p in procs:
         p.start()
-    res = [q.get(timeout=300) for _ in range(2)]
+    res = [q.get(timeout=300) for _ in range(world)]
     for p in procs:
         p.join(timeout=120)
         assert p.exitcode == 0
