@@ -313,9 +313,10 @@ AFD_API afd_status_t afd_ffn_route_noalloc(const afd_ffn_config_t* cfg, const af
  * into this device's address space (peer pointers), and several plans, on this or other
  * GPUs, may add into the same buffers at the same time. The buffers must hold zeros where
  * rows will be added before the first such call (afd_combine_finalize leaves them zero).
- * NULL restores the plan's own accumulators and the bf16 slab outputs. Copies the table
- * to the device (synchronous). AFD_ERR_INVALID_ARGUMENT for a NULL plan, a NULL or
- * misaligned entry, or a current device other than the plan's.
+ * NULL restores the plan's own accumulators and the bf16 slab outputs. The plan keeps a
+ * copy of the table and passes it with every down-projection launch (nothing is written
+ * to the device; the host array may be freed after the call). AFD_ERR_INVALID_ARGUMENT
+ * for a NULL plan, a NULL or misaligned entry, or a current device other than the plan's.
  *
  * afd_combine_finalize: on the GPU of the owning attention rank, once every FFN GPU's
  * additions have completed: for each of num_slabs slabs and t < counts[m], writes
